@@ -1,0 +1,183 @@
+"""CPU oracle for MoE token-to-expert routing (test infrastructure only).
+
+This package is the slow, plain reference that the CUDA library is checked
+against.  Only the tests, the smoke check and the CPU-baseline leg of the
+benchmark may import it; the product package never does.  It shares no code
+with the CUDA path: the arithmetic lives in ``moe_routing_oracle.c`` (plain C,
+double precision, one row at a time) and this module only compiles it with
+gcc and marshals numpy arrays into it.
+
+Operations (each a restatement of the SGLang MoE routing page,
+"[SGLang] MoE 라우팅: 토큰에서 전문가로의 배분 알고리즘"):
+
+* :func:`topk_softmax`        - §2 softmax top-k (optional renormalise)
+* :func:`grouped_topk`        - §3 grouped top-k, group score = max
+* :func:`biased_grouped_topk` - §4 sigmoid + correction_bias, group score =
+  sum of the top-2 biased scores; with num_expert_group = topk_group = 1 it is
+  the sigmoid top-k of the aiter page ("SGLang MoE 라우팅 최적화: AMD GPU에서
+  aiter.biased_grouped_topk 활용", 코드 분석)
+* :func:`router_logits`       - §5 router projection, exact products summed
+  in double
+* :func:`fused_router_topk`   - §5 projection followed by §4 routing
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_routing_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+SOFTMAX, SIGMOID = 0, 1
+GROUP_MAX, GROUP_TOP2_SUM = 0, 1
+
+_DBL = ctypes.POINTER(ctypes.c_double)
+_I32 = ctypes.POINTER(ctypes.c_int32)
+
+
+def compile_oracle(src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the C oracle into a shared library with gcc (IEEE double, no
+    fast-math, no FMA contraction).  Returns the library path."""
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off",
+           "-fno-fast-math", "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    lib.oracle_route.restype = ctypes.c_int
+    lib.oracle_route.argtypes = [
+        _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, _DBL, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+        _I32, _DBL, _DBL, _DBL, _DBL]
+    lib.oracle_router_logits.restype = ctypes.c_int
+    lib.oracle_router_logits.argtypes = [
+        _DBL, _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _DBL]
+    return lib
+
+
+def load(path: str | None = None):
+    """Load (compiling first if needed) the oracle library."""
+    global _lib
+    if path is not None:
+        return _bind(path)
+    with _lock:
+        if _lib is None:
+            if (not os.path.exists(_LIB_PATH)
+                    or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+                compile_oracle()
+            _lib = _bind(_LIB_PATH)
+    return _lib
+
+
+def as_f64(a) -> np.ndarray:
+    """Exact conversion of stored input values (numpy, or a CPU torch tensor of
+    any float dtype including bfloat16) to a C-contiguous float64 array."""
+    if hasattr(a, "detach"):
+        import torch  # local: only needed when handed a tensor
+        a = a.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a, ty):
+    return None if a is None else a.ctypes.data_as(ty)
+
+
+class Routing:
+    """Result of one oracle call (all numpy)."""
+
+    def __init__(self, ids, weights, sel, gsc, margins):
+        self.ids = ids          # (M, k) int32
+        self.weights = weights  # (M, k) float64
+        self.sel = sel          # (M, E) float64 selection scores
+        self.group_scores = gsc  # (M, G) float64
+        self.margins = margins  # (M, 3) float64: expert, group, selected-gap
+
+
+def route(logits, *, scoring: int, bias=None, num_expert_group: int = 1,
+          topk_group: int = 1, group_kind: int = GROUP_MAX, topk: int,
+          renormalize: bool, routed_scaling_factor: float = 1.0,
+          lib=None) -> Routing:
+    x = as_f64(logits)
+    if x.ndim != 2:
+        raise ValueError("logits must be 2-D (M, E)")
+    M, E = x.shape
+    b = None if bias is None else as_f64(bias).reshape(E)
+    G = int(num_expert_group)
+    ids = np.zeros((M, topk), dtype=np.int32)
+    w = np.zeros((M, topk), dtype=np.float64)
+    sel = np.zeros((M, E), dtype=np.float64)
+    gsc = np.zeros((M, G), dtype=np.float64)
+    mg = np.zeros((M, 3), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_route(_ptr(x, _DBL), M, E, scoring, _ptr(b, _DBL), G,
+                          int(topk_group), group_kind, int(topk), int(bool(renormalize)),
+                          float(routed_scaling_factor), _ptr(ids, _I32), _ptr(w, _DBL),
+                          _ptr(sel, _DBL), _ptr(gsc, _DBL), _ptr(mg, _DBL))
+    if rc == 1:
+        raise ValueError("oracle_route: invalid arguments")
+    if rc != 0:
+        raise MemoryError("oracle_route: out of memory")
+    return Routing(ids, w, sel, gsc, mg)
+
+
+def topk_softmax(logits, topk: int, renormalize: bool, lib=None) -> Routing:
+    return route(logits, scoring=SOFTMAX, topk=topk, renormalize=renormalize,
+                 group_kind=GROUP_MAX, lib=lib)
+
+
+def grouped_topk(logits, topk: int, renormalize: bool, num_expert_group: int,
+                 topk_group: int, routed_scaling_factor: float = 1.0, lib=None) -> Routing:
+    return route(logits, scoring=SOFTMAX, topk=topk, renormalize=renormalize,
+                 num_expert_group=num_expert_group, topk_group=topk_group,
+                 group_kind=GROUP_MAX, routed_scaling_factor=routed_scaling_factor,
+                 lib=lib)
+
+
+def biased_grouped_topk(logits, correction_bias, topk: int, renormalize: bool,
+                        num_expert_group: int, topk_group: int,
+                        routed_scaling_factor: float = 1.0, lib=None) -> Routing:
+    return route(logits, scoring=SIGMOID, bias=correction_bias, topk=topk,
+                 renormalize=renormalize, num_expert_group=num_expert_group,
+                 topk_group=topk_group, group_kind=GROUP_TOP2_SUM,
+                 routed_scaling_factor=routed_scaling_factor, lib=lib)
+
+
+def router_logits(hidden_states, router_weight, *, weight_layout: int = 0,
+                  lib=None) -> np.ndarray:
+    """logits = hidden_states x W.  weight_layout 0: W is (K, E); 1: W is (E, K)."""
+    h = as_f64(hidden_states)
+    w = as_f64(router_weight)
+    M, K = h.shape
+    E = w.shape[1] if weight_layout == 0 else w.shape[0]
+    if (weight_layout == 0 and w.shape[0] != K) or (weight_layout == 1 and w.shape[1] != K):
+        raise ValueError("router_weight shape does not match hidden_states")
+    out = np.zeros((M, E), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_router_logits(_ptr(h, _DBL), _ptr(w, _DBL), M, K, E, int(weight_layout),
+                                  _ptr(out, _DBL))
+    if rc != 0:
+        raise ValueError("oracle_router_logits: invalid arguments")
+    return out
+
+
+def fused_router_topk(hidden_states, router_weight, correction_bias, topk: int,
+                      renormalize: bool, num_expert_group: int, topk_group: int,
+                      routed_scaling_factor: float = 1.0, weight_layout: int = 0,
+                      lib=None):
+    """Projection then biased grouped top-k.  Returns (Routing, logits)."""
+    logits = router_logits(hidden_states, router_weight, weight_layout=weight_layout, lib=lib)
+    r = biased_grouped_topk(logits, correction_bias, topk, renormalize, num_expert_group,
+                            topk_group, routed_scaling_factor, lib=lib)
+    return r, logits

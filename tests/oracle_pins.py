@@ -1,0 +1,228 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each check takes an oracle library handle and returns a list of failure
+strings (empty = pass), so the same checks can be run against the real
+oracle (tests/test_oracle_pins.py) and against deliberately broken copies of
+its source (tests/test_oracle_mutants.py), proving that a plausible slip in
+the oracle would be caught.
+
+Pins used:
+* golden hand-worked cases (tests/golden/*.json, closed forms, each cited);
+* brute force: the kept groups are the topk_group-subset with the largest
+  total group score, and the picks are the k-subset of admissible experts
+  with the largest total selection score (unique for distinct values);
+* library cross-checks for the ungrouped cases: scipy's softmax / expit and a
+  stable numpy argsort reproduce the scores, ids and weights;
+* the router projection against numpy's float64 matmul and a hand case.
+"""
+from __future__ import annotations
+
+import glob
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+from scipy.special import expit, softmax
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _logits_from(case):
+    if case["logits_from"] == "ln(u)":
+        return np.log(np.asarray(case["u"], dtype=np.float64))[None, :]
+    if case["logits_from"] == "logit(p)":
+        p = np.asarray(case["p"], dtype=np.float64)
+        return np.log(p / (1.0 - p))[None, :]
+    raise ValueError(case["logits_from"])
+
+
+def _run_case(case, lib):
+    x = _logits_from(case)
+    op = case["op"]
+    if op == "topk_softmax":
+        return oracle.topk_softmax(x, case["topk"], case["renormalize"], lib=lib)
+    if op == "grouped_topk":
+        return oracle.grouped_topk(x, case["topk"], case["renormalize"], case["num_expert_group"],
+                                   case["topk_group"], case["routed_scaling_factor"], lib=lib)
+    if op == "biased_grouped_topk":
+        return oracle.biased_grouped_topk(x, np.asarray(case["bias"], np.float64), case["topk"],
+                                          case["renormalize"], case["num_expert_group"],
+                                          case["topk_group"], case["routed_scaling_factor"],
+                                          lib=lib)
+    raise ValueError(op)
+
+
+def check_golden(lib) -> list[str]:
+    fails = []
+    for path in sorted(glob.glob(os.path.join(GOLDEN, "*_e8.json"))):
+        doc = json.load(open(path))
+        for n, case in enumerate(doc["cases"]):
+            try:
+                r = _run_case(case, lib)
+            except Exception as exc:  # a broken oracle may reject valid args
+                fails.append(f"{os.path.basename(path)}[{n}]: raised {exc!r}")
+                continue
+            if r.ids[0].tolist() != case["ids"]:
+                fails.append(f"{os.path.basename(path)}[{n}]: ids {r.ids[0].tolist()} != {case['ids']}")
+            if not np.allclose(r.weights[0], case["weights"], rtol=0, atol=1e-12):
+                fails.append(f"{os.path.basename(path)}[{n}]: weights {r.weights[0]} != {case['weights']}")
+    return fails
+
+
+def check_router_golden(lib) -> list[str]:
+    doc = json.load(open(os.path.join(GOLDEN, "router_logits_small.json")))
+    h = np.asarray(doc["hidden"], np.float64)
+    w = np.asarray(doc["weight_ke"], np.float64)
+    fails = []
+    got = oracle.router_logits(h, w, weight_layout=0, lib=lib)
+    if not np.array_equal(got, np.asarray(doc["logits"])):
+        fails.append(f"router (K,E) hand case: {got.tolist()}")
+    got_t = oracle.router_logits(h, np.ascontiguousarray(w.T), weight_layout=1, lib=lib)
+    if not np.array_equal(got_t, np.asarray(doc["logits"])):
+        fails.append(f"router (E,K) hand case: {got_t.tolist()}")
+    return fails
+
+
+def check_router_numpy(lib, seed=7) -> list[str]:
+    rng = np.random.default_rng(seed)
+    h = rng.standard_normal((5, 37))
+    w = rng.standard_normal((37, 11))
+    ref = h @ w
+    fails = []
+    for layout, wt in ((0, w), (1, np.ascontiguousarray(w.T))):
+        got = oracle.router_logits(h, wt, weight_layout=layout, lib=lib)
+        if not np.allclose(got, ref, rtol=1e-12, atol=1e-12):
+            fails.append(f"router layout {layout}: max err {np.abs(got - ref).max()}")
+    return fails
+
+
+# --------------------------------------------------------------------------
+# brute force over subsets
+# --------------------------------------------------------------------------
+def _brute(s, G, TG, k, group_kind):
+    """Independent formulation: best TG-subset of groups by total group score,
+    then the best k-subset of their experts by total selection score."""
+    E = len(s)
+    S = E // G
+    gs = []
+    for g in range(G):
+        vals = sorted(s[g * S:(g + 1) * S], reverse=True)
+        gs.append(vals[0] if group_kind == oracle.GROUP_MAX else sum(vals[:2]))
+    best_groups = max(itertools.combinations(range(G), TG), key=lambda c: sum(gs[g] for g in c))
+    adm = [e for e in range(E) if e // S in best_groups]
+    best = max(itertools.combinations(adm, k), key=lambda c: sum(s[e] for e in c))
+    return set(best_groups), set(best)
+
+
+def check_brute(lib, trials=150, seed=11) -> list[str]:
+    rng = np.random.default_rng(seed)
+    fails = []
+    shapes = [(8, 1, 1, 2), (8, 4, 2, 3), (8, 2, 1, 4), (12, 3, 2, 5), (12, 4, 3, 4),
+              (12, 6, 2, 3), (10, 5, 4, 6), (9, 3, 1, 3), (6, 6, 3, 3), (12, 12, 5, 5)]
+    for t in range(trials):
+        E, G, TG, k = shapes[t % len(shapes)]
+        x = rng.standard_normal((1, E)) * 2.0
+        kind = t % 3
+        if kind == 0:   # softmax, group max
+            r = oracle.grouped_topk(x, k, True, G, TG, lib=lib)
+            p = softmax(x[0])
+            s = p
+            gk = oracle.GROUP_MAX
+        else:           # sigmoid + bias, sum of top-2
+            b = rng.standard_normal(E) * (0.3 if kind == 1 else 0.0)
+            r = oracle.biased_grouped_topk(x, b, k, True, G, TG, lib=lib)
+            p = expit(x[0])
+            s = p + b
+            gk = oracle.GROUP_TOP2_SUM
+        _, picks = _brute(list(s), G, TG, k, gk)
+        got = r.ids[0].tolist()
+        if set(got) != picks:
+            fails.append(f"brute t={t} E={E} G={G} TG={TG} k={k}: {sorted(got)} != {sorted(picks)}")
+            continue
+        if any(s[got[j]] < s[got[j + 1]] for j in range(k - 1)):
+            fails.append(f"brute t={t}: ids not in descending score order")
+        w = p[got]
+        w = w / w.sum()
+        if not np.allclose(r.weights[0], w, rtol=1e-12, atol=1e-15):
+            fails.append(f"brute t={t}: weights {r.weights[0]} != {w}")
+    return fails
+
+
+# --------------------------------------------------------------------------
+# library cross-checks (ungrouped cases reduce to a stable sort)
+# --------------------------------------------------------------------------
+def _stable_topk(s, k):
+    # stable sort on -s: equal scores keep ascending index order
+    return np.argsort(-s, kind="stable")[:k]
+
+
+def check_library(lib, seed=5) -> list[str]:
+    rng = np.random.default_rng(seed)
+    fails = []
+    # softmax top-k, E=64, with and without renormalise
+    x = rng.standard_normal((40, 64)) * 1.5
+    for renorm in (False, True):
+        r = oracle.topk_softmax(x, 6, renorm, lib=lib)
+        for i in range(x.shape[0]):
+            p = softmax(x[i])
+            ids = _stable_topk(p, 6)
+            w = p[ids] / (p[ids].sum() if renorm else 1.0)
+            if r.ids[i].tolist() != ids.tolist():
+                fails.append(f"softmax row {i}: ids {r.ids[i]} != {ids}")
+                break
+            if not np.allclose(r.weights[i], w, rtol=1e-12, atol=1e-15):
+                fails.append(f"softmax row {i}: weights")
+                break
+    # sigmoid + bias, one group (the aiter form), scaled
+    x = rng.standard_normal((40, 96)) * 2.0
+    b = rng.standard_normal(96) * 0.05
+    r = oracle.biased_grouped_topk(x, b, 8, True, 1, 1, 2.5, lib=lib)
+    for i in range(x.shape[0]):
+        p = expit(x[i])
+        ids = _stable_topk(p + b, 8)
+        w = 2.5 * p[ids] / p[ids].sum()
+        if r.ids[i].tolist() != ids.tolist():
+            fails.append(f"sigmoid row {i}: ids {r.ids[i]} != {ids}")
+            break
+        if not np.allclose(r.weights[i], w, rtol=1e-12, atol=1e-15):
+            fails.append(f"sigmoid row {i}: weights")
+            break
+    # no bias, no renormalise: weights are the plain sigmoid scores
+    r = oracle.biased_grouped_topk(x, None, 5, False, 1, 1, lib=lib)
+    for i in range(x.shape[0]):
+        p = expit(x[i])
+        ids = _stable_topk(p, 5)
+        if r.ids[i].tolist() != ids.tolist() or not np.allclose(r.weights[i], p[ids], rtol=1e-12):
+            fails.append(f"plain sigmoid row {i}")
+            break
+    # grouping with every group kept (TG == G) equals the ungrouped result
+    x = rng.standard_normal((20, 32))
+    a = oracle.grouped_topk(x, 4, True, 8, 8, lib=lib)
+    c = oracle.topk_softmax(x, 4, True, lib=lib)
+    if not (np.array_equal(a.ids, c.ids) and np.allclose(a.weights, c.weights, rtol=1e-14)):
+        fails.append("TG == G differs from ungrouped")
+    # margins: the expert margin is the gap between the k-th and (k+1)-th score
+    r = oracle.biased_grouped_topk(x, None, 4, True, 1, 1, lib=lib)
+    for i in range(x.shape[0]):
+        srt = np.sort(expit(x[i]))[::-1]
+        if not math.isclose(r.margins[i, 0], srt[3] - srt[4], rel_tol=1e-12, abs_tol=1e-15):
+            fails.append(f"margin row {i}")
+            break
+    return fails
+
+
+ALL_CHECKS = (check_golden, check_router_golden, check_router_numpy, check_brute, check_library)
+
+
+def run_all(lib) -> list[str]:
+    fails = []
+    for chk in ALL_CHECKS:
+        try:
+            fails += chk(lib)
+        except Exception as exc:
+            fails.append(f"{chk.__name__} raised {exc!r}")
+    return fails

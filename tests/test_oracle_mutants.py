@@ -1,0 +1,59 @@
+"""Plausible slips in the oracle are caught by the pins.
+
+Each mutant is a copy of the oracle's C source with one deliberate mistake
+(a dropped term, a wrong sign or index, a transposed operand, a flipped
+tie-break ...).  It is compiled into a temporary directory on the CPU and the
+pin suite must report at least one failure for it (or the mutant must
+crash, which a pin run would also expose).  The real oracle source is
+never modified.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_routing_oracle.c")
+
+MUTANTS = {
+    "bias_sign": ("s[e] = p[e] + (bias ? bias[e] : 0.0);", "s[e] = p[e] - (bias ? bias[e] : 0.0);"),
+    "gather_biased": ("weights[i * (int64_t)k + j] = p[admissible[j].index];",
+                      "weights[i * (int64_t)k + j] = s[admissible[j].index];"),
+    "drop_second_in_top2": ("return best + second;", "return best;"),
+    "tie_higher_index": ("if (a->index < b->index) return -1;\n    if (a->index > b->index) return 1;",
+                         "if (a->index < b->index) return 1;\n    if (a->index > b->index) return -1;"),
+    "sigmoid_sign": ("p[e] = 1.0 / (1.0 + exp(-x[e]));", "p[e] = 1.0 / (1.0 + exp(x[e]));"),
+    "skip_best_group": ("for (int t = 0; t < TG; ++t) group_kept", "for (int t = 1; t < TG; ++t) group_kept"),
+    "no_renorm": ("if (renorm) w = w / wsum;", "if (0) w = w / wsum;"),
+    "scale_divides": ("weights[i * (int64_t)k + j] = w * rsf;", "weights[i * (int64_t)k + j] = w / rsf;"),
+    "softmax_sign": ("p[e] = exp(x[e] - mx);", "p[e] = exp(mx - x[e]);"),
+    "softmax_unnormalised": ("for (int e = 0; e < E; ++e) p[e] = p[e] / sum;", ";"),
+    "interleaved_groups": ("if (group_kept[e / S]) {", "if (group_kept[e % G]) {"),
+    "transposed_weight": ("double wv = (w_layout == 0) ? w[(int64_t)c * E + e] : w[(int64_t)e * K + c];",
+                          "double wv = (w_layout == 0) ? w[(int64_t)e * K + c] : w[(int64_t)c * E + e];"),
+    "ascending_order": ("if (a->value > b->value) return -1;\n    if (a->value < b->value) return 1;",
+                        "if (a->value > b->value) return 1;\n    if (a->value < b->value) return -1;"),
+    "group_max_is_min": ("if (s[first + j] > m) m = s[first + j];", "if (s[first + j] < m) m = s[first + j];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mutant_src = tmp_path / f"mutant_{name}.c"
+    mutant_src.write_text(src.replace(old, new))
+    so = oracle.compile_oracle(str(mutant_src), str(tmp_path / f"libmutant_{name}.so"))
+    # Run the pins in a child process: a mutant may also crash (an index
+    # slip can read out of bounds), which counts as caught.
+    code = ("import sys, oracle; from tests import oracle_pins; "
+            f"f = oracle_pins.run_all(oracle.load({str(so)!r})); "
+            "print(len(f)); sys.exit(0 if f else 3)")
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                         timeout=300)
+    assert res.returncode != 3, f"mutant {name} passed every pin"
