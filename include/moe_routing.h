@@ -1,0 +1,189 @@
+/*
+ * moe_routing.h - C ABI of the B200 (sm_100a) Mixture-of-Experts
+ * token-to-expert routing library (libmoe_routing.so).
+ *
+ * Every entry point routes M token rows of router logits to k experts each and
+ * writes, per row, k expert ids (int32) and k routing weights (fp32):
+ *
+ *   scores      softmax over the row, or sigmoid per expert
+ *   choice      selection score = score + correction_bias (bias optional)
+ *   groups      the E experts form num_expert_group contiguous groups of
+ *               S = E / num_expert_group; each group gets a score (its largest
+ *               selection score, or the sum of its two largest); the
+ *               topk_group best groups are kept and every expert of the other
+ *               groups is excluded
+ *   top-k       the k best selection scores among the kept experts
+ *   weights     the UNBIASED scores of the chosen experts; if renormalize,
+ *               divided by their sum; then multiplied by routed_scaling_factor
+ *
+ * Sources (pages on SGLang MoE routing, cited by title and section):
+ *   [R] "[SGLang] MoE 라우팅: 토큰에서 전문가로의 배분 알고리즘"
+ *       §2 기본 softmax Top-K, §3 Grouped Top-K, §4 Biased Grouped Top-K,
+ *       §5 Fused MoE Router; the fused_topk / grouped_topk_gpu /
+ *       biased_grouped_topk_impl signatures shown there
+ *   [A] "[sglang] SGLang MoE 라우팅 최적화: AMD GPU에서 aiter.biased_grouped_topk 활용",
+ *       코드 분석 (After): the aiter_biased_grouped_topk call with
+ *       num_expert_group=1, topk_group=1, need_renorm=renormalize
+ *
+ * Conventions shared by every call
+ *   - Tie-break: between equal selection scores (and equal group scores) the
+ *     lower index wins.  Ids are written in descending selection score, ties in
+ *     ascending index.  (The pages leave this open; this is the reading taken.)
+ *   - Layout: every matrix is row-major and densely packed (row stride = number
+ *     of columns).  Outputs are (M, topk) row-major.
+ *   - Memory: all pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees, synchronises or prints.  Calls are asynchronous
+ *     on `stream` (a cudaStream_t passed as void*, NULL = legacy default
+ *     stream) and may be captured in a CUDA graph.
+ *   - Errors: the return value is a moe_status_t.  Invalid arguments are
+ *     rejected before anything is launched (MOE_ERR_INVALID_ARG); shapes the
+ *     library was not built for give MOE_ERR_UNSUPPORTED; a failed launch gives
+ *     MOE_ERR_CUDA.  moe_last_error() returns a message for the calling thread's
+ *     last failure.  M == 0 is valid and launches nothing.
+ *   - Inputs must be finite; NaN or infinity in the logits is outside the
+ *     contract (no per-element check is made; the output is then unspecified
+ *     but every written id is still in [0, E)).
+ *   - Arithmetic is fp32 on the device from bf16 or fp32 inputs.
+ */
+#ifndef MOE_ROUTING_H
+#define MOE_ROUTING_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ROUTING_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* argument outside the documented domain     */
+    MOE_ERR_UNSUPPORTED = 2, /* valid, but this build has no kernel for it */
+    MOE_ERR_CUDA = 3         /* the CUDA runtime reported an error         */
+} moe_status_t;
+
+typedef enum {
+    MOE_DTYPE_F32 = 0,
+    MOE_DTYPE_BF16 = 1
+} moe_dtype_t;
+
+typedef enum {
+    MOE_WEIGHT_K_BY_E = 0, /* router weight stored (K, E): hidden x W        */
+    MOE_WEIGHT_E_BY_K = 1  /* router weight stored (E, K): nn.Linear layout  */
+} moe_weight_layout_t;
+
+/* Library ABI version (MOE_ROUTING_ABI_VERSION of the build). */
+MOE_API int moe_abi_version(void);
+
+/* Static text for a status code. */
+MOE_API const char* moe_status_string(int status);
+
+/* Message describing the calling thread's most recent non-OK return. */
+MOE_API const char* moe_last_error(void);
+
+/*
+ * moe_topk_softmax - [R] §2: softmax over each row, top-k, optional
+ * renormalise (the sgl_kernel topk_softmax(topk_weights, topk_ids,
+ * gating_output, renormalize) call).
+ *
+ *   gating_output  device, (M, E) of `dtype` (MOE_DTYPE_F32 or MOE_DTYPE_BF16)
+ *   M              rows, M >= 0
+ *   E              experts, 1 <= E <= 1024
+ *   topk           1 <= topk <= min(E, 32)
+ *   renormalize    nonzero: weights divided by their sum
+ *   topk_weights   device, (M, topk) fp32 out
+ *   topk_ids       device, (M, topk) int32 out
+ *   stream         cudaStream_t
+ */
+MOE_API int moe_topk_softmax(const void* gating_output, int dtype, int64_t M, int32_t E,
+                     int32_t topk, int32_t renormalize, float* topk_weights,
+                     int32_t* topk_ids, void* stream);
+
+/*
+ * moe_grouped_topk - [R] §3 (DeepSeek-V2 grouped_topk_gpu): softmax scores,
+ * group score = the group's largest score, keep the topk_group best groups,
+ * top-k over their experts, optional renormalise, then scale.
+ *
+ *   num_expert_group  G >= 1, G divides E
+ *   topk_group        1 <= topk_group <= G
+ *   topk              1 <= topk <= min(topk_group * E / G, 32)
+ *   routed_scaling_factor  finite multiplier applied last (1.0 = none)
+ *   other arguments as moe_topk_softmax
+ */
+MOE_API int moe_grouped_topk(const void* gating_output, int dtype, int64_t M, int32_t E,
+                     int32_t topk, int32_t renormalize, int32_t num_expert_group,
+                     int32_t topk_group, float routed_scaling_factor,
+                     float* topk_weights, int32_t* topk_ids, void* stream);
+
+/*
+ * moe_biased_grouped_topk - [R] §4 (DeepSeek-V3 biased_grouped_topk_impl) and
+ * [A] (aiter biased_grouped_topk): sigmoid scores; selection score = score +
+ * correction_bias; group score = sum of the group's two largest selection
+ * scores (a one-expert group: that score); keep the topk_group best groups;
+ * top-k by selection score; weights are the unbiased sigmoid scores,
+ * optionally renormalised, then scaled.  num_expert_group = topk_group = 1 is
+ * the plain sigmoid(+bias) top-k of sgl_kernel topk_sigmoid.
+ *
+ *   correction_bias  device, (E,) fp32, or NULL for no bias.  It stays fp32
+ *                    (the aiter path casts it to the logits dtype; this
+ *                    library does not).
+ *   other arguments as moe_grouped_topk
+ */
+MOE_API int moe_biased_grouped_topk(const void* gating_output, int dtype,
+                            const float* correction_bias, int64_t M, int32_t E,
+                            int32_t topk, int32_t renormalize,
+                            int32_t num_expert_group, int32_t topk_group,
+                            float routed_scaling_factor, float* topk_weights,
+                            int32_t* topk_ids, void* stream);
+
+/*
+ * moe_fused_router_workspace_size - bytes of device workspace that
+ * moe_fused_router_topk needs for these sizes (0 when it needs none).
+ * Returns (size_t)-1 for arguments moe_fused_router_topk would reject.
+ */
+MOE_API size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E);
+
+/*
+ * moe_fused_router_topk - [R] §5 (FusedMoeRouter) with the [R] §4 routing:
+ * logits = hidden_states x router_weight accumulated in fp32 on the tensor
+ * cores and kept on chip, then the moe_biased_grouped_topk routing of those
+ * logits.  The logits never reach device memory unless logits_out is given.
+ *
+ *   hidden_states   device, (M, K) bf16
+ *   router_weight   device, bf16, (K, E) if weight_layout == MOE_WEIGHT_K_BY_E
+ *                   or (E, K) if MOE_WEIGHT_E_BY_K
+ *   correction_bias device, (E,) fp32, or NULL
+ *   K               hidden size, a positive multiple of 64
+ *   E               experts; this build supports E == 256
+ *   logits_out      device, (M, E) fp32 out, or NULL (debug: the fp32 logits
+ *                   the routing consumed)
+ *   workspace       device scratch of at least
+ *                   moe_fused_router_workspace_size(M, K, E) bytes, 256-byte
+ *                   aligned (NULL allowed when that size is 0).  Its contents
+ *                   need no initialisation and are left in a state that the
+ *                   next call accepts; calls that overlap on the GPU must not
+ *                   share one workspace.
+ *   other arguments as moe_biased_grouped_topk
+ */
+MOE_API int moe_fused_router_topk(const void* hidden_states, const void* router_weight,
+                          int weight_layout, const float* correction_bias,
+                          int64_t M, int32_t K, int32_t E, int32_t topk,
+                          int32_t renormalize, int32_t num_expert_group,
+                          int32_t topk_group, float routed_scaling_factor,
+                          float* topk_weights, int32_t* topk_ids,
+                          float* logits_out, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_ROUTING_H */

@@ -1,0 +1,24 @@
+"""B200-native (sm_100a) Mixture-of-Experts token-to-expert routing.
+
+The compute lives in ``libmoe_routing.so`` (hand-written CUDA kernels behind
+the C ABI in ``include/moe_routing.h``); this package is its thin binding.
+Build the library with ``python -m moe_expert_routing_token_b200.build``.
+"""
+from .routing import (  # noqa: F401
+    MOE_DTYPE_BF16,
+    MOE_DTYPE_F32,
+    MOE_WEIGHT_E_BY_K,
+    MOE_WEIGHT_K_BY_E,
+    RoutingError,
+    biased_grouped_topk,
+    fused_router_topk,
+    fused_router_workspace_size,
+    grouped_topk,
+    lib,
+    topk_softmax,
+)
+
+__all__ = [
+    "topk_softmax", "grouped_topk", "biased_grouped_topk", "fused_router_topk",
+    "fused_router_workspace_size", "lib", "RoutingError",
+]

@@ -1,0 +1,259 @@
+// C ABI of libmoe_routing: argument validation, kernel choice and launch.
+//
+// Calls follow the signatures of the SGLang routing pages: fused_topk /
+// topk_softmax (softmax top-k), grouped_topk_gpu (grouped top-k),
+// biased_grouped_topk_impl and aiter_biased_grouped_topk (sigmoid +
+// correction_bias), FusedMoeRouter (router projection + routing).  Nothing
+// here allocates, synchronises or prints, so every call can be captured in a
+// CUDA graph.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <unordered_map>
+
+#include "fused_router.cuh"
+#include "moe_routing.h"
+#include "routing_kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+thread_local char g_last_error[512] = "no error";
+
+int fail(int status, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int cuda_fail(cudaError_t err, const char* what) {
+    return fail(MOE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(err), cudaGetErrorString(err));
+}
+
+// Per-device SM count and per-kernel residency, looked up once.
+struct LaunchCache {
+    std::mutex mu;
+    std::unordered_map<int, int> sms;
+    std::unordered_map<const void*, int> per_sm[64];
+};
+LaunchCache& cache() {
+    static LaunchCache c;
+    return c;
+}
+
+int device_and_sms(int* dev, int* sms) {
+    cudaError_t err = cudaGetDevice(dev);
+    if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
+    LaunchCache& c = cache();
+    std::lock_guard<std::mutex> lk(c.mu);
+    auto it = c.sms.find(*dev);
+    if (it != c.sms.end()) {
+        *sms = it->second;
+        return MOE_OK;
+    }
+    int n = 0;
+    err = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, *dev);
+    if (err != cudaSuccess) return cuda_fail(err, "cudaDeviceGetAttribute");
+    c.sms[*dev] = n;
+    *sms = n;
+    return MOE_OK;
+}
+
+template <typename Kernel>
+int resident_blocks(int dev, Kernel k, int threads, size_t smem, int* out) {
+    LaunchCache& c = cache();
+    const void* key = reinterpret_cast<const void*>(k);
+    std::lock_guard<std::mutex> lk(c.mu);
+    auto& m = c.per_sm[dev & 63];
+    auto it = m.find(key);
+    if (it != m.end()) {
+        *out = it->second;
+        return MOE_OK;
+    }
+    int n = 0;
+    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem);
+    if (err != cudaSuccess) return cuda_fail(err, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (n < 1) n = 1;
+    m[key] = n;
+    *out = n;
+    return MOE_OK;
+}
+
+// Persistent-style grid: enough blocks for the work, capped at one full wave
+// of resident blocks over all SMs.
+template <typename Kernel>
+int launch_rows(Kernel k, int threads, size_t smem, int64_t rows_per_block, const RouteArgs& a,
+                cudaStream_t stream) {
+    int dev = 0, sms = 0, per_sm = 1;
+    int rc = device_and_sms(&dev, &sms);
+    if (rc != MOE_OK) return rc;
+    rc = resident_blocks(dev, k, threads, smem, &per_sm);
+    if (rc != MOE_OK) return rc;
+    const int64_t need = (a.M + rows_per_block - 1) / rows_per_block;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const int grid = (int)(need < cap ? need : cap);
+    k<<<grid, threads, smem, stream>>>(a);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "routing kernel launch");
+    return MOE_OK;
+}
+
+bool aligned(const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+template <typename TIn, int SCORE, bool BIAS>
+int launch_segment(int E, const RouteArgs& a, cudaStream_t st) {
+    if (E == 256) {
+        constexpr int L = 256 / 32, R = 32 / L;
+        return launch_rows(route_segment_kernel<TIn, 256, 32, SCORE, BIAS>, kSegThreads, 0,
+                           (kSegThreads / 32) * R, a, st);
+    }
+    constexpr int L = 160 / 20, R = 32 / L;
+    return launch_rows(route_segment_kernel<TIn, 160, 20, SCORE, BIAS>, kSegThreads, 0,
+                       (kSegThreads / 32) * R, a, st);
+}
+
+template <typename TIn, int SCORE, bool BIAS>
+int launch_small(int E, const RouteArgs& a, cudaStream_t st) {
+    switch (E) {
+        case 8: return launch_rows(route_small_kernel<TIn, 8, SCORE, BIAS>, 256, 0, 256, a, st);
+        case 16: return launch_rows(route_small_kernel<TIn, 16, SCORE, BIAS>, 256, 0, 256, a, st);
+        default: return launch_rows(route_small_kernel<TIn, 32, SCORE, BIAS>, 256, 0, 256, a, st);
+    }
+}
+
+template <typename TIn, int SCORE>
+int launch_generic(const RouteArgs& a, cudaStream_t st) {
+    const int per_warp = generic_smem_per_warp(a.E, a.G);
+    int warps = (48 * 1024) / per_warp;
+    if (warps > 4) warps = 4;
+    if (warps < 1) return fail(MOE_ERR_UNSUPPORTED, "E=%d, G=%d need too much shared memory", a.E, a.G);
+    return launch_rows(route_generic_kernel<TIn, SCORE>, warps * 32, (size_t)warps * per_warp,
+                       warps, a, st);
+}
+
+template <typename TIn, int SCORE, bool BIAS>
+int dispatch_typed(const RouteArgs& a, cudaStream_t st) {
+    const int E = a.E;
+    const size_t esz = sizeof(TIn);
+    if ((E == 256 || E == 160) && (E == 256 ? 8 : 8) % a.G == 0) {
+        const int C = (E == 256) ? 32 : 20;
+        const size_t chunk = C * esz;
+        const size_t vec = (chunk % 16 == 0) ? 16 : 8;
+        if (aligned(a.logits, vec)) return launch_segment<TIn, SCORE, BIAS>(E, a, st);
+    }
+    if ((E == 8 || E == 16 || E == 32) && aligned(a.logits, 16))
+        return launch_small<TIn, SCORE, BIAS>(E, a, st);
+    return launch_generic<TIn, SCORE>(a, st);
+}
+
+int route(const void* logits, int dtype, const float* bias, int64_t M, int E, int K, int renorm,
+          int G, int TG, int group_kind, int scoring, float rsf, float* weights, int32_t* ids,
+          void* stream, const char* who) {
+    if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16)
+        return fail(MOE_ERR_INVALID_ARG, "%s: dtype %d is neither MOE_DTYPE_F32 nor MOE_DTYPE_BF16", who, dtype);
+    if (M < 0) return fail(MOE_ERR_INVALID_ARG, "%s: M=%lld < 0", who, (long long)M);
+    if (E < 1) return fail(MOE_ERR_INVALID_ARG, "%s: E=%d < 1", who, E);
+    if (G < 1 || E % G != 0)
+        return fail(MOE_ERR_INVALID_ARG, "%s: num_expert_group=%d does not divide E=%d", who, G, E);
+    if (TG < 1 || TG > G)
+        return fail(MOE_ERR_INVALID_ARG, "%s: topk_group=%d outside [1, %d]", who, TG, G);
+    if (K < 1 || K > TG * (E / G))
+        return fail(MOE_ERR_INVALID_ARG, "%s: topk=%d outside [1, topk_group*E/G=%d]", who, K, TG * (E / G));
+    if (!std::isfinite(rsf)) return fail(MOE_ERR_INVALID_ARG, "%s: routed_scaling_factor is not finite", who);
+    if (E > 1024) return fail(MOE_ERR_UNSUPPORTED, "%s: E=%d > 1024", who, E);
+    if (K > 32) return fail(MOE_ERR_UNSUPPORTED, "%s: topk=%d > 32", who, K);
+    if (M == 0) return MOE_OK;
+    if (!logits || !weights || !ids) return fail(MOE_ERR_INVALID_ARG, "%s: null pointer argument", who);
+    const size_t esz = dtype == MOE_DTYPE_F32 ? 4 : 2;
+    if (!aligned(logits, esz) || !aligned(weights, 4) || !aligned(ids, 4) || (bias && !aligned(bias, 4)))
+        return fail(MOE_ERR_INVALID_ARG, "%s: pointer not aligned to its element size", who);
+
+    RouteArgs a;
+    a.logits = logits;
+    a.bias = bias;
+    a.M = M;
+    a.E = E;
+    a.G = G;
+    a.TG = TG;
+    a.K = K;
+    a.group_kind = group_kind;
+    a.renorm = renorm ? 1 : 0;
+    a.rsf = rsf;
+    a.weights = weights;
+    a.ids = ids;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (scoring == kSoftmax) {
+        a.bias = nullptr;
+        return dtype == MOE_DTYPE_F32 ? dispatch_typed<float, kSoftmax, false>(a, st)
+                                      : dispatch_typed<__nv_bfloat16, kSoftmax, false>(a, st);
+    }
+    if (bias)
+        return dtype == MOE_DTYPE_F32 ? dispatch_typed<float, kSigmoid, true>(a, st)
+                                      : dispatch_typed<__nv_bfloat16, kSigmoid, true>(a, st);
+    return dtype == MOE_DTYPE_F32 ? dispatch_typed<float, kSigmoid, false>(a, st)
+                                  : dispatch_typed<__nv_bfloat16, kSigmoid, false>(a, st);
+}
+
+}  // namespace
+
+int set_error(int status, const char* msg) { return fail(status, "%s", msg); }
+int set_cuda_error(cudaError_t err, const char* what) { return cuda_fail(err, what); }
+int sm_count(int* dev, int* sms) { return device_and_sms(dev, sms); }
+int route_logits(const void* logits, int dtype, const float* bias, int64_t M, int E, int K,
+                 int renorm, int G, int TG, float rsf, float* weights, int32_t* ids, void* stream) {
+    return route(logits, dtype, bias, M, E, K, renorm, G, TG, kGroupTop2Sum, kSigmoid, rsf, weights,
+                 ids, stream, "moe_fused_router_topk");
+}
+
+}  // namespace moe
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ROUTING_ABI_VERSION; }
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+const char* moe_last_error(void) { return moe::g_last_error; }
+
+int moe_topk_softmax(const void* gating_output, int dtype, int64_t M, int32_t E, int32_t topk,
+                     int32_t renormalize, float* topk_weights, int32_t* topk_ids, void* stream) {
+    return moe::route(gating_output, dtype, nullptr, M, E, topk, renormalize, 1, 1, moe::kGroupMax,
+                      moe::kSoftmax, 1.0f, topk_weights, topk_ids, stream, "moe_topk_softmax");
+}
+
+int moe_grouped_topk(const void* gating_output, int dtype, int64_t M, int32_t E, int32_t topk,
+                     int32_t renormalize, int32_t num_expert_group, int32_t topk_group,
+                     float routed_scaling_factor, float* topk_weights, int32_t* topk_ids,
+                     void* stream) {
+    return moe::route(gating_output, dtype, nullptr, M, E, topk, renormalize, num_expert_group,
+                      topk_group, moe::kGroupMax, moe::kSoftmax, routed_scaling_factor, topk_weights,
+                      topk_ids, stream, "moe_grouped_topk");
+}
+
+int moe_biased_grouped_topk(const void* gating_output, int dtype, const float* correction_bias,
+                            int64_t M, int32_t E, int32_t topk, int32_t renormalize,
+                            int32_t num_expert_group, int32_t topk_group,
+                            float routed_scaling_factor, float* topk_weights, int32_t* topk_ids,
+                            void* stream) {
+    return moe::route(gating_output, dtype, correction_bias, M, E, topk, renormalize,
+                      num_expert_group, topk_group, moe::kGroupTop2Sum, moe::kSigmoid,
+                      routed_scaling_factor, topk_weights, topk_ids, stream,
+                      "moe_biased_grouped_topk");
+}
+
+}  // extern "C"

@@ -1,0 +1,456 @@
+// Routing kernels: logits (M, E) -> topk_weights (M, K) fp32, topk_ids (M, K) int32.
+//
+// What they compute is the routing of the SGLang MoE routing page
+// ("[SGLang] MoE 라우팅: 토큰에서 전문가로의 배분 알고리즘"): §2 softmax top-k,
+// §3 grouped top-k (group score = max) and §4 biased grouped top-k (sigmoid +
+// correction_bias, group score = sum of the top-2 biased scores), with the
+// gathered weights being the unbiased scores, renormalised and scaled.  Ties
+// go to the lower expert / group index and ids leave in descending score.
+//
+// Three kernels, picked by shape:
+//
+//  * route_segment_kernel (the hot path, E = 160 or 256): a row is owned by a
+//    segment of L = E / C lanes, each lane holding C consecutive experts in
+//    registers after one pass of 16-byte loads.  A lane's chunk never
+//    straddles a group, so group scores need only xor-shuffles among the
+//    group's lanes.  Instead of k rounds of arg-max, the kernel derives a
+//    threshold tau that the k-th best admissible score is known to reach (the
+//    ceil(k/2)-th best per-lane second-largest score among kept lanes: those
+//    lanes alone hold k admissible experts >= tau), collects the few
+//    candidates >= tau into shared memory, and ranks each candidate by
+//    counting how many candidates beat it - the ballot/popcount rank idea of
+//    the MiniMax-M3 page's warp rank sort, applied to scores.  Rows with more
+//    than kCandCap candidates (massive ties) take an exact k-round arg-max.
+//  * route_small_kernel (E <= 32): one thread per row, k rounds of arg-max in
+//    registers.
+//  * route_generic_kernel (any E <= 1024, any group shape, any alignment): one
+//    warp per row, row staged in shared memory, k rounds of warp arg-max.
+#pragma once
+
+#include "routing_common.cuh"
+
+namespace moe {
+
+constexpr int kSegThreads = 128;
+constexpr int kCandCap = 32;
+
+__device__ __forceinline__ unsigned seg_bits(int L) { return L >= 32 ? kFullMask : ((1u << L) - 1u); }
+
+template <typename TIn, int E, int C, int SCORE, bool BIAS>
+__global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a) {
+    constexpr int L = E / C;   // lanes per row
+    constexpr int R = 32 / L;  // rows per warp
+    constexpr int WARPS = kSegThreads / 32;
+    constexpr int CQ = (C / 4) | 1;  // odd number of float4 per lane: conflict-free STS.128
+    constexpr int CS = CQ * 4;
+    constexpr int TPL = (32 + L - 1) / L;  // output ranks per lane (k <= 32)
+    static_assert(E % C == 0 && 32 % L == 0 && C % 4 == 0 && C <= 32, "bad segment shape");
+
+    __shared__ __align__(16) float s_p[WARPS][R * L * CS];  // unbiased score (softmax: logit)
+    __shared__ float2 s_cand[WARPS][R][kCandCap + 1];     // candidate (key, id)
+    __shared__ float s_candp[WARPS][R][kCandCap];         // candidate unbiased score
+    __shared__ float2 s_out[WARPS][R][32];                // by rank: (score, id)
+    __shared__ float s_bias[BIAS ? E : 1];
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int seg = lane / L;
+    const int sl = lane % L;
+    const int base = seg * L;
+    const int e0 = sl * C;
+
+    float b_r[C];
+    if constexpr (BIAS) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) s_bias[e] = __ldg(a.bias + e);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < C; ++i) b_r[i] = s_bias[e0 + i];
+    }
+
+    const int G = a.G, TG = a.TG, K = a.K;
+    const int P = L / G;  // lanes per group (the dispatcher guarantees G | L)
+    const int g = sl / P;
+    const bool all_groups = (TG == G);
+    const int nsel_lanes = all_groups ? L : TG * P;
+    const int need = (K + 1) >> 1;
+    const unsigned smask = seg_bits(L) << base;
+
+    float* my_p = &s_p[warp][(seg * L + sl) * CS];
+    const TIn* logits = static_cast<const TIn*>(a.logits);
+    const int64_t step = (int64_t)gridDim.x * WARPS * R;
+
+    for (int64_t row0 = ((int64_t)blockIdx.x * WARPS + warp) * R; row0 < a.M; row0 += step) {
+        const int64_t row = row0 + seg;
+        const bool valid = row < a.M;
+
+        float x[C];
+        if (valid) {
+            ChunkLoader<TIn, C>::load(logits + row * E + e0, x);
+        } else {
+#pragma unroll
+            for (int i = 0; i < C; ++i) x[i] = 0.0f;
+        }
+
+        // Pass 1: score, selection key, per-lane top-2 of the keys.
+        float key[C];
+        float m1 = -INFINITY, m2 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+            const float p = (SCORE == kSigmoid) ? sigmoid_f32(x[i]) : x[i];
+            x[i] = p;
+            key[i] = BIAS ? p + b_r[i] : p;
+            top2_push(m1, m2, key[i]);
+        }
+#pragma unroll
+        for (int q = 0; q < C / 4; ++q)
+            reinterpret_cast<float4*>(my_p)[q] =
+                make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+
+        // Group score from the group's lanes, then keep the TG best groups.
+        float g1 = m1, g2 = m2;
+        for (int o = 1; o < P; o <<= 1) {
+            const float b1 = __shfl_xor_sync(kFullMask, g1, o);
+            const float b2 = __shfl_xor_sync(kFullMask, g2, o);
+            top2_merge(g1, g2, b1, b2);
+        }
+        const float gs = (a.group_kind == kGroupTop2Sum) ? g1 + g2 : g1;
+        bool gsel = true;
+        if (!all_groups) {
+            int rank = 0;
+            for (int h = 0; h < G; ++h) {
+                const float o = __shfl_sync(kFullMask, gs, base + h * P);
+                rank += (o > gs) || (o == gs && h < g);
+            }
+            gsel = rank < TG;
+        }
+
+        // Threshold: the kept lanes with the `need` largest second-best keys
+        // hold at least K admissible experts with key >= tau.
+        float tau;
+        if (need > nsel_lanes) {
+            tau = -INFINITY;
+        } else if (need == nsel_lanes) {
+            float v = gsel ? m2 : INFINITY;
+#pragma unroll
+            for (int o = L / 2; o >= 1; o >>= 1) v = fminf(v, __shfl_xor_sync(kFullMask, v, o));
+            tau = v;
+        } else {
+            const float my = gsel ? m2 : -INFINITY;
+            int r = 0;
+#pragma unroll
+            for (int j = 0; j < L; ++j) {
+                const float o = __shfl_sync(kFullMask, my, base + j);
+                r += (o > my) || (o == my && j < sl);
+            }
+            const unsigned bal = __ballot_sync(kFullMask, r == need - 1) & smask;
+            tau = __shfl_sync(kFullMask, my, __ffs(bal) - 1);
+        }
+
+        // Candidates: kept experts with key >= tau.
+        unsigned mask = 0u;
+        if (gsel) {
+#pragma unroll
+            for (int i = 0; i < C; ++i) mask |= (key[i] >= tau ? 1u : 0u) << i;
+        }
+        const int cnt = __popc(mask);
+        int n = cnt;
+#pragma unroll
+        for (int o = L / 2; o >= 1; o >>= 1) n += __shfl_xor_sync(kFullMask, n, o);
+
+        const bool exact_needed = valid && (n > kCandCap || n < K);
+        if (__any_sync(kFullMask, exact_needed)) {
+            // Exact K rounds of segment arg-max (massive ties; rare).
+            unsigned taken = 0u;
+            for (int j = 0; j < K; ++j) {
+                int bi = -1;
+                float bv = -INFINITY;
+                if (gsel) {
+#pragma unroll
+                    for (int i = 0; i < C; ++i)
+                        if (!((taken >> i) & 1u) && (bi < 0 || key[i] > bv)) {
+                            bv = key[i];
+                            bi = i;
+                        }
+                }
+                float wv = bi < 0 ? -INFINITY : bv;
+                int wi = bi < 0 ? 0x7fffffff : e0 + bi;
+#pragma unroll
+                for (int o = L / 2; o >= 1; o >>= 1) {
+                    const float ov = __shfl_xor_sync(kFullMask, wv, o);
+                    const int oi = __shfl_xor_sync(kFullMask, wi, o);
+                    if (beats(ov, oi, wv, wi)) {
+                        wv = ov;
+                        wi = oi;
+                    }
+                }
+                if (bi >= 0 && wi == e0 + bi) taken |= 1u << bi;
+                if (sl == 0) {
+                    const int gi = (wi >= 0 && wi < E) ? wi : 0;
+                    s_out[warp][seg][j] =
+                        make_float2(s_p[warp][(seg * L + gi / C) * CS + gi % C], __int_as_float(gi));
+                }
+            }
+            __syncwarp();
+        } else {
+            // Compact the candidates of the segment into shared memory ...
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < L; o <<= 1) {
+                const int t = __shfl_up_sync(kFullMask, incl, o);
+                if (sl >= o) incl += t;
+            }
+            int pos = incl - cnt;
+            unsigned mm = valid ? mask : 0u;
+            while (mm) {
+                const int b = __ffs(mm) - 1;
+                mm &= mm - 1u;
+                const float pv = my_p[b];
+                const float kv = BIAS ? pv + s_bias[e0 + b] : pv;
+                s_cand[warp][seg][pos] = make_float2(kv, __int_as_float(e0 + b));
+                s_candp[warp][seg][pos] = pv;
+                ++pos;
+            }
+            __syncwarp();
+            // ... and rank each one by counting the candidates that beat it.
+            const int nn = valid ? n : 0;
+            for (int t = sl; t < nn; t += L) {
+                const float2 c = s_cand[warp][seg][t];
+                const int ci = __float_as_int(c.y);
+                int r = 0;
+                for (int u = 0; u < nn; ++u) {
+                    const float2 d = s_cand[warp][seg][u];
+                    r += beats(d.x, __float_as_int(d.y), c.x, ci) ? 1 : 0;
+                }
+                if (r < K) s_out[warp][seg][r] = make_float2(s_candp[warp][seg][t], c.y);
+            }
+            __syncwarp();
+        }
+
+        // Weights: gather the unbiased scores, renormalise, scale.
+        float rowmax = 0.0f, denom_all = 1.0f;
+        if constexpr (SCORE == kSoftmax) {
+            float mx = m1;
+#pragma unroll
+            for (int o = L / 2; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, o));
+            rowmax = mx;
+            if (!a.renorm) {
+                float s = 0.0f;
+#pragma unroll
+                for (int i = 0; i < C; ++i) s += exp_f32(key[i] - rowmax);
+#pragma unroll
+                for (int o = L / 2; o >= 1; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
+                denom_all = s;
+            }
+        }
+        float w_loc[TPL];
+        int id_loc[TPL];
+        float sum = 0.0f;
+#pragma unroll
+        for (int q = 0; q < TPL; ++q) {
+            const int t = sl + q * L;
+            w_loc[q] = 0.0f;
+            id_loc[q] = 0;
+            if (t < K) {
+                const float2 o = s_out[warp][seg][t];
+                const float w = (SCORE == kSoftmax) ? exp_f32(o.x - rowmax) : o.x;
+                w_loc[q] = w;
+                id_loc[q] = __float_as_int(o.y);
+                sum += w;
+            }
+        }
+        float scale;
+        if (a.renorm) {
+#pragma unroll
+            for (int o = L / 2; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
+            scale = a.rsf / sum;
+        } else {
+            scale = (SCORE == kSoftmax) ? a.rsf / denom_all : a.rsf;
+        }
+        if (valid) {
+#pragma unroll
+            for (int q = 0; q < TPL; ++q) {
+                const int t = sl + q * L;
+                if (t < K) {
+                    a.weights[row * K + t] = w_loc[q] * scale;
+                    a.ids[row * K + t] = id_loc[q];
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// One thread per row, E <= 32.
+// ---------------------------------------------------------------------------
+template <typename TIn, int E, int SCORE, bool BIAS>
+__global__ void __launch_bounds__(256) route_small_kernel(RouteArgs a) {
+    const TIn* logits = static_cast<const TIn*>(a.logits);
+    const int G = a.G, TG = a.TG, K = a.K;
+    const int S = E / G;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; row < a.M; row += stride) {
+        float x[E];
+        ChunkLoader<TIn, E>::load(logits + row * E, x);
+        float p[E], key[E];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            p[i] = (SCORE == kSigmoid) ? sigmoid_f32(x[i]) : x[i];
+            key[i] = BIAS ? p[i] + __ldg(a.bias + i) : p[i];
+            mx = fmaxf(mx, x[i]);
+        }
+        // admissible experts: those of the TG best groups
+        unsigned adm = (E >= 32) ? kFullMask : ((1u << E) - 1u);
+        if (TG < G) {
+            float gs[E];
+#pragma unroll
+            for (int h = 0; h < E; ++h) gs[h] = -INFINITY;
+            for (int h = 0; h < G; ++h) {
+                float t1 = -INFINITY, t2 = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < E; ++i)
+                    if (i / S == h) top2_push(t1, t2, key[i]);
+                gs[h] = (a.group_kind == kGroupTop2Sum) ? t1 + t2 : t1;
+            }
+            unsigned gmask = 0u;
+            for (int h = 0; h < G; ++h) {
+                int rank = 0;
+                for (int o = 0; o < G; ++o) rank += beats(gs[o], o, gs[h], h) ? 1 : 0;
+                if (rank < TG) gmask |= 1u << h;
+            }
+            adm = 0u;
+#pragma unroll
+            for (int i = 0; i < E; ++i)
+                if ((gmask >> (i / S)) & 1u) adm |= 1u << i;
+        }
+        float denom_all = 1.0f;
+        if (SCORE == kSoftmax && !a.renorm) {
+            float s = 0.0f;
+#pragma unroll
+            for (int i = 0; i < E; ++i) s += exp_f32(x[i] - mx);
+            denom_all = s;
+        }
+        float sum = 0.0f;
+        unsigned taken = 0u;
+        for (int j = 0; j < K; ++j) {
+            int bi = -1;
+            float bv = -INFINITY, bp = 0.0f;
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                if (((adm & ~taken) >> i) & 1u) {
+                    if (bi < 0 || key[i] > bv) {
+                        bv = key[i];
+                        bi = i;
+                        bp = p[i];
+                    }
+                }
+            }
+            if (bi < 0) bi = 0;  // unreachable for valid arguments
+            taken |= 1u << bi;
+            const float w = (SCORE == kSoftmax) ? exp_f32(bp - mx) : bp;
+            sum += w;
+            a.weights[row * K + j] = w;
+            a.ids[row * K + j] = bi;
+        }
+        const float scale = a.renorm ? a.rsf / sum : ((SCORE == kSoftmax) ? a.rsf / denom_all : a.rsf);
+        for (int j = 0; j < K; ++j) a.weights[row * K + j] *= scale;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// One warp per row, any E <= 1024, any group shape, scalar loads.
+// Dynamic shared memory per warp: 2*E floats + G floats + E bytes, 16-aligned.
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr int generic_smem_per_warp(int E, int G) {
+    return ((2 * E + G) * 4 + E + 15) / 16 * 16;
+}
+
+template <typename TIn, int SCORE>
+__global__ void __launch_bounds__(128) route_generic_kernel(RouteArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int E = a.E, G = a.G, TG = a.TG, K = a.K;
+    const int S = E / G;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int warps = blockDim.x >> 5;
+    unsigned char* wbase = smem + (size_t)warp * generic_smem_per_warp(E, G);
+    float* s_p = reinterpret_cast<float*>(wbase);
+    float* s_key = s_p + E;
+    float* s_gs = s_key + E;
+    unsigned char* s_flag = reinterpret_cast<unsigned char*>(s_gs + G);  // bit0 kept, bit1 taken
+    const TIn* logits = static_cast<const TIn*>(a.logits);
+
+    for (int64_t row = (int64_t)blockIdx.x * warps + warp; row < a.M; row += (int64_t)gridDim.x * warps) {
+        float mx = -INFINITY;
+        for (int e = lane; e < E; e += 32) {
+            const float x = load_scalar<TIn>(logits + row * E + e);
+            const float p = (SCORE == kSigmoid) ? sigmoid_f32(x) : x;
+            s_p[e] = p;
+            s_key[e] = (a.bias != nullptr) ? p + __ldg(a.bias + e) : p;
+            mx = fmaxf(mx, x);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, o));
+        __syncwarp();
+        for (int h = lane; h < G; h += 32) {
+            float t1 = -INFINITY, t2 = -INFINITY;
+            for (int j = 0; j < S; ++j) top2_push(t1, t2, s_key[h * S + j]);
+            s_gs[h] = (a.group_kind == kGroupTop2Sum && S > 1) ? t1 + t2 : t1;
+        }
+        __syncwarp();
+        for (int h = lane; h < G; h += 32) {
+            int rank = 0;
+            for (int o = 0; o < G; ++o) rank += beats(s_gs[o], o, s_gs[h], h) ? 1 : 0;
+            const unsigned char kept = (TG >= G || rank < TG) ? 1 : 0;
+            for (int j = 0; j < S; ++j) s_flag[h * S + j] = kept;
+        }
+        __syncwarp();
+        float denom_all = 1.0f;
+        if (SCORE == kSoftmax && !a.renorm) {
+            float s = 0.0f;
+            for (int e = lane; e < E; e += 32) s += exp_f32(s_p[e] - mx);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
+            denom_all = s;
+        }
+        float sum = 0.0f, my_w = 0.0f;
+        int my_id = 0;
+        for (int j = 0; j < K; ++j) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int e = lane; e < E; e += 32)
+                if (s_flag[e] == 1 && (bi == 0x7fffffff || beats(s_key[e], e, bv, bi))) {
+                    bv = s_key[e];
+                    bi = e;
+                }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const float ov = __shfl_xor_sync(kFullMask, bv, o);
+                const int oi = __shfl_xor_sync(kFullMask, bi, o);
+                if ((oi != 0x7fffffff && bi == 0x7fffffff) || (oi != 0x7fffffff && beats(ov, oi, bv, bi))) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            if (bi == 0x7fffffff) bi = 0;  // unreachable for valid arguments
+            const float w = (SCORE == kSoftmax) ? exp_f32(s_p[bi] - mx) : s_p[bi];
+            sum += w;
+            if (lane == j) {
+                my_w = w;
+                my_id = bi;
+            }
+            __syncwarp();
+            if (lane == 0) s_flag[bi] = 3;
+            __syncwarp();
+        }
+        const float scale = a.renorm ? a.rsf / sum : ((SCORE == kSoftmax) ? a.rsf / denom_all : a.rsf);
+        if (lane < K) {
+            a.weights[row * K + lane] = my_w * scale;
+            a.ids[row * K + lane] = my_id;
+        }
+        __syncwarp();
+    }
+}
+
+}  // namespace moe

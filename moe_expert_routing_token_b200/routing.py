@@ -1,0 +1,209 @@
+"""Thin Python binding of libmoe_routing (argument marshalling only).
+
+Every function here checks tensor placement, dtype and layout, allocates the
+outputs the way SGLang's ``fused_topk`` does (``torch.empty`` of (M, k) fp32
+weights and int32 ids), and calls the matching C entry point of
+``include/moe_routing.h`` with raw device pointers and the current CUDA
+stream.  All routing arithmetic runs in the library's CUDA kernels; there is
+no CPU or PyTorch fallback - if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libmoe_routing.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 0, 1, 2, 3
+MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
+MOE_WEIGHT_K_BY_E, MOE_WEIGHT_E_BY_K = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_f32 = ctypes.c_float
+_sz = ctypes.c_size_t
+
+SIGNATURES = {
+    "moe_abi_version": (ctypes.c_int, []),
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_last_error": (ctypes.c_char_p, []),
+    "moe_topk_softmax": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_grouped_topk": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _i32, _i32, _i32, _i32, _f32,
+                                        _vp, _vp, _vp]),
+    "moe_biased_grouped_topk": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32, _i32,
+                                               _i32, _f32, _vp, _vp, _vp]),
+    "moe_fused_router_workspace_size": (_sz, [_i64, _i32, _i32]),
+    "moe_fused_router_topk": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32, _i32,
+                                             _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+}
+
+
+class RoutingError(RuntimeError):
+    """A CUDA-side failure reported by libmoe_routing."""
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"libmoe_routing.so not found at {LIB_PATH}; build it with "
+                    "`python -m moe_expert_routing_token_b200.build`")
+            handle = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(handle, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = handle
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status == MOE_OK:
+        return
+    msg = lib().moe_last_error().decode()
+    if status == MOE_ERR_INVALID_ARG:
+        raise ValueError(f"{what}: {msg}")
+    if status == MOE_ERR_UNSUPPORTED:
+        raise NotImplementedError(f"{what}: {msg}")
+    raise RoutingError(f"{what}: {msg}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MOE_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_DTYPE_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}; expected float32 or bfloat16")
+
+
+def _cuda_2d(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 2-D tensor")
+
+
+def _bias_ptr(bias, E: int, device) -> int | None:
+    if bias is None:
+        return None
+    if not bias.is_cuda or bias.device != device or bias.dtype != torch.float32:
+        raise ValueError("correction_bias must be a float32 CUDA tensor on the logits' device")
+    if bias.numel() != E or not bias.is_contiguous():
+        raise ValueError("correction_bias must be a contiguous (E,) tensor")
+    return bias.data_ptr()
+
+
+def _outputs(M: int, topk: int, device, out):
+    if out is not None:
+        w, ids = out
+        if (w.shape != (M, topk) or w.dtype != torch.float32 or ids.shape != (M, topk)
+                or ids.dtype != torch.int32 or not w.is_contiguous() or not ids.is_contiguous()
+                or w.device != device or ids.device != device):
+            raise ValueError("out must be ((M, topk) float32, (M, topk) int32) contiguous on the device")
+        return w, ids
+    return (torch.empty(M, topk, dtype=torch.float32, device=device),
+            torch.empty(M, topk, dtype=torch.int32, device=device))
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def topk_softmax(gating_output: torch.Tensor, topk: int, renormalize: bool, out=None):
+    """Softmax top-k of each row.  Returns (topk_weights fp32, topk_ids int32)."""
+    _cuda_2d(gating_output, "gating_output")
+    M, E = gating_output.shape
+    w, ids = _outputs(M, topk, gating_output.device, out)
+    st = lib().moe_topk_softmax(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
+                                int(bool(renormalize)), w.data_ptr(), ids.data_ptr(),
+                                _stream(gating_output.device))
+    _check(st, "moe_topk_softmax")
+    return w, ids
+
+
+def grouped_topk(gating_output: torch.Tensor, topk: int, renormalize: bool, num_expert_group: int,
+                 topk_group: int, routed_scaling_factor: float = 1.0, out=None):
+    """Softmax grouped top-k (group score = max).  Returns (weights, ids)."""
+    _cuda_2d(gating_output, "gating_output")
+    M, E = gating_output.shape
+    w, ids = _outputs(M, topk, gating_output.device, out)
+    st = lib().moe_grouped_topk(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
+                                int(bool(renormalize)), num_expert_group, topk_group,
+                                float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
+                                _stream(gating_output.device))
+    _check(st, "moe_grouped_topk")
+    return w, ids
+
+
+def biased_grouped_topk(gating_output: torch.Tensor, correction_bias, topk: int,
+                        renormalize: bool, num_expert_group: int = 1, topk_group: int = 1,
+                        routed_scaling_factor: float = 1.0, out=None):
+    """Sigmoid + correction_bias grouped top-k (group score = sum of top-2).
+    With num_expert_group = topk_group = 1 it is the sigmoid top-k."""
+    _cuda_2d(gating_output, "gating_output")
+    M, E = gating_output.shape
+    bp = _bias_ptr(correction_bias, E, gating_output.device)
+    w, ids = _outputs(M, topk, gating_output.device, out)
+    st = lib().moe_biased_grouped_topk(gating_output.data_ptr(), _dtype_code(gating_output), bp, M, E,
+                                       topk, int(bool(renormalize)), num_expert_group, topk_group,
+                                       float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
+                                       _stream(gating_output.device))
+    _check(st, "moe_biased_grouped_topk")
+    return w, ids
+
+
+def fused_router_workspace_size(M: int, K: int, E: int) -> int:
+    n = lib().moe_fused_router_workspace_size(M, K, E)
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("moe_fused_router_workspace_size: invalid sizes")
+    return n
+
+
+def fused_router_topk(hidden_states: torch.Tensor, router_weight: torch.Tensor, correction_bias,
+                      topk: int, renormalize: bool, num_expert_group: int, topk_group: int,
+                      routed_scaling_factor: float = 1.0, weight_layout: str = "ke",
+                      return_logits: bool = False, workspace: torch.Tensor | None = None, out=None):
+    """Router projection on the tensor cores fused with biased grouped top-k.
+
+    ``weight_layout`` "ke": router_weight is (K, E); "ek": (E, K).  Returns
+    (weights, ids) or (weights, ids, logits fp32) with ``return_logits``.
+    """
+    _cuda_2d(hidden_states, "hidden_states")
+    _cuda_2d(router_weight, "router_weight")
+    if hidden_states.dtype != torch.bfloat16 or router_weight.dtype != torch.bfloat16:
+        raise ValueError("hidden_states and router_weight must be bfloat16")
+    M, K = hidden_states.shape
+    if weight_layout == "ke":
+        layout, (Kw, E) = MOE_WEIGHT_K_BY_E, router_weight.shape
+    elif weight_layout == "ek":
+        layout, (E, Kw) = MOE_WEIGHT_E_BY_K, router_weight.shape
+    else:
+        raise ValueError("weight_layout must be 'ke' or 'ek'")
+    if Kw != K:
+        raise ValueError("router_weight does not match hidden_states' hidden size")
+    dev = hidden_states.device
+    bp = _bias_ptr(correction_bias, E, dev)
+    w, ids = _outputs(M, topk, dev, out)
+    logits = torch.empty(M, E, dtype=torch.float32, device=dev) if return_logits else None
+    need = fused_router_workspace_size(M, K, E)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wsp = workspace.data_ptr() if (need and workspace is not None) else None
+    st = lib().moe_fused_router_topk(hidden_states.data_ptr(), router_weight.data_ptr(), layout, bp, M,
+                                     K, E, topk, int(bool(renormalize)), num_expert_group, topk_group,
+                                     float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
+                                     None if logits is None else logits.data_ptr(), wsp,
+                                     need if wsp else 0, _stream(dev))
+    _check(st, "moe_fused_router_topk")
+    return (w, ids, logits) if return_logits else (w, ids)

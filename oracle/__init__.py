@@ -60,7 +60,7 @@ def _bind(path: str):
     lib.oracle_route.argtypes = [
         _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, _DBL, ctypes.c_int,
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-        _I32, _DBL, _DBL, _DBL, _DBL]
+        _I32, _DBL, _DBL, _DBL, _DBL, _DBL]
     lib.oracle_router_logits.restype = ctypes.c_int
     lib.oracle_router_logits.argtypes = [
         _DBL, _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _DBL]
@@ -97,9 +97,10 @@ def _ptr(a, ty):
 class Routing:
     """Result of one oracle call (all numpy)."""
 
-    def __init__(self, ids, weights, sel, gsc, margins):
+    def __init__(self, ids, weights, scores, sel, gsc, margins):
         self.ids = ids          # (M, k) int32
         self.weights = weights  # (M, k) float64
+        self.scores = scores    # (M, E) float64 unbiased scores
         self.sel = sel          # (M, E) float64 selection scores
         self.group_scores = gsc  # (M, G) float64
         self.margins = margins  # (M, 3) float64: expert, group, selected-gap
@@ -117,6 +118,7 @@ def route(logits, *, scoring: int, bias=None, num_expert_group: int = 1,
     G = int(num_expert_group)
     ids = np.zeros((M, topk), dtype=np.int32)
     w = np.zeros((M, topk), dtype=np.float64)
+    scores = np.zeros((M, E), dtype=np.float64)
     sel = np.zeros((M, E), dtype=np.float64)
     gsc = np.zeros((M, G), dtype=np.float64)
     mg = np.zeros((M, 3), dtype=np.float64)
@@ -124,12 +126,12 @@ def route(logits, *, scoring: int, bias=None, num_expert_group: int = 1,
     rc = lib.oracle_route(_ptr(x, _DBL), M, E, scoring, _ptr(b, _DBL), G,
                           int(topk_group), group_kind, int(topk), int(bool(renormalize)),
                           float(routed_scaling_factor), _ptr(ids, _I32), _ptr(w, _DBL),
-                          _ptr(sel, _DBL), _ptr(gsc, _DBL), _ptr(mg, _DBL))
+                          _ptr(scores, _DBL), _ptr(sel, _DBL), _ptr(gsc, _DBL), _ptr(mg, _DBL))
     if rc == 1:
         raise ValueError("oracle_route: invalid arguments")
     if rc != 0:
         raise MemoryError("oracle_route: out of memory")
-    return Routing(ids, w, sel, gsc, mg)
+    return Routing(ids, w, scores, sel, gsc, mg)
 
 
 def topk_softmax(logits, topk: int, renormalize: bool, lib=None) -> Routing:

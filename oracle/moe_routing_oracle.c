@@ -132,6 +132,7 @@ static double group_score(const double* s, int first, int S, int kind) {
  * Outputs (row-major):
  *   ids      M x k   expert ids, descending selection score
  *   weights  M x k   the gathered unbiased scores after renorm and scaling
+ *   scores   M x E   unbiased scores p (NULL to skip)
  *   sel      M x E   selection scores s = p + bias (NULL to skip)
  *   gsc      M x G   group scores (NULL to skip)
  *   margins  M x 3   [0] s_(k) - s_(k+1) over the admissible experts
@@ -145,7 +146,7 @@ static double group_score(const double* s, int first, int S, int kind) {
 int oracle_route(const double* logits, int64_t M, int E, int scoring,
                  const double* bias, int G, int TG, int group_kind, int k,
                  int renorm, double rsf, int32_t* ids, double* weights,
-                 double* sel, double* gsc, double* margins) {
+                 double* scores, double* sel, double* gsc, double* margins) {
     if (M < 0 || E < 1 || G < 1 || E % G != 0 || TG < 1 || TG > G || k < 1)
         return ORACLE_BAD_ARGS;
     const int S = E / G;
@@ -169,6 +170,8 @@ int oracle_route(const double* logits, int64_t M, int E, int scoring,
 
         /* 1. scores */
         score_row(x, E, scoring, p);
+        if (scores)
+            for (int e = 0; e < E; ++e) scores[i * (int64_t)E + e] = p[e];
 
         /* 2. selection scores: bias steers the choice only ([R] §4) */
         for (int e = 0; e < E; ++e) s[e] = p[e] + (bias ? bias[e] : 0.0);

@@ -24,3 +24,12 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionstart(session):
+    # Build the CUDA library and the oracle once per test session (no-ops when
+    # they are up to date).  Building needs nvcc but no GPU.
+    from moe_expert_routing_token_b200 import build
+    build.build()
+    import oracle
+    oracle.load()

@@ -1,0 +1,94 @@
+"""The C-ABI library loads, exports every declared symbol and validates its
+arguments on the host (CPU only: no compute call needs a GPU here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import moe_expert_routing_token_b200 as moe
+from moe_expert_routing_token_b200 import routing
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_routing.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return moe.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ("moe_topk_softmax", "moe_grouped_topk", "moe_biased_grouped_topk",
+              "moe_fused_router_topk", "moe_fused_router_workspace_size"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert name in routing.SIGNATURES, f"binding lacks {name}"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.moe_abi_version() == 1
+    assert lib.moe_status_string(0) == b"MOE_OK"
+    assert lib.moe_status_string(1) == b"MOE_ERR_INVALID_ARG"
+    assert lib.moe_status_string(2) == b"MOE_ERR_UNSUPPORTED"
+    assert lib.moe_status_string(3) == b"MOE_ERR_CUDA"
+
+
+# Host-side validation returns before any CUDA call, so it runs without a GPU.
+P = 4096  # a non-null dummy address; never dereferenced on these paths
+
+
+@pytest.mark.parametrize("args,status,needle", [
+    # moe_grouped_topk(logits, dtype, M, E, topk, renorm, G, TG, rsf, w, ids, stream)
+    ((P, 0, 4, 8, 2, 1, 3, 1, 1.0, P, P, None), 1, "does not divide"),
+    ((P, 0, 4, 8, 2, 1, 4, 5, 1.0, P, P, None), 1, "topk_group"),
+    ((P, 0, 4, 8, 2, 1, 4, 0, 1.0, P, P, None), 1, "topk_group"),
+    ((P, 0, 4, 8, 5, 1, 4, 2, 1.0, P, P, None), 1, "topk=5"),
+    ((P, 0, 4, 8, 0, 1, 4, 2, 1.0, P, P, None), 1, "topk=0"),
+    ((P, 7, 4, 8, 2, 1, 4, 2, 1.0, P, P, None), 1, "dtype"),
+    ((P, 0, -1, 8, 2, 1, 4, 2, 1.0, P, P, None), 1, "M=-1"),
+    ((P, 0, 4, 0, 2, 1, 1, 1, 1.0, P, P, None), 1, "E=0"),
+    ((P, 0, 4, 8, 2, 1, 4, 2, float("nan"), P, P, None), 1, "scaling"),
+    ((None, 0, 4, 8, 2, 1, 4, 2, 1.0, P, P, None), 1, "null"),
+    ((P, 0, 4, 8, 2, 1, 4, 2, 1.0, None, P, None), 1, "null"),
+    ((P + 2, 0, 4, 8, 2, 1, 4, 2, 1.0, P, P, None), 1, "aligned"),
+    ((P, 0, 4, 2048, 2, 1, 1, 1, 1.0, P, P, None), 2, "E=2048"),
+    ((P, 0, 4, 64, 33, 1, 1, 1, 1.0, P, P, None), 2, "topk=33"),
+])
+def test_grouped_topk_validation(lib, args, status, needle):
+    assert lib.moe_grouped_topk(*args) == status
+    assert needle in lib.moe_last_error().decode()
+
+
+def test_empty_batch_is_ok_without_launch(lib):
+    assert lib.moe_topk_softmax(None, 0, 0, 8, 2, 1, None, None, None) == 0
+    assert lib.moe_biased_grouped_topk(None, 1, None, 0, 256, 8, 1, 8, 4, 2.5, None, None, None) == 0
+
+
+def test_biased_validation(lib):
+    # bias pointer not 4-byte aligned
+    assert lib.moe_biased_grouped_topk(P, 1, P + 1, 4, 256, 8, 1, 8, 4, 2.5, P, P, None) == 1
+    assert lib.moe_biased_grouped_topk(P, 1, None, 4, 256, 8, 1, 8, 9, 2.5, P, P, None) == 1
+
+
+def test_fused_router_workspace_query(lib):
+    assert lib.moe_fused_router_workspace_size(-1, 7168, 256) == ctypes.c_size_t(-1).value
+    n = lib.moe_fused_router_workspace_size(64, 7168, 256)
+    assert n != ctypes.c_size_t(-1).value
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 8)
+    with pytest.raises(ValueError):
+        moe.topk_softmax(x, 2, True)

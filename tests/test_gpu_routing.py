@@ -1,0 +1,203 @@
+"""CUDA routing kernels against the CPU oracle (GPU only).
+
+Every call goes through the C ABI (via the thin binding).  Covers the four
+routing workloads at their quoted token counts (the full sizes, in the same
+launch configuration the benchmark times), ragged and tiny batches, dtype
+variants, every kernel family (segment / small-E / generic), massive ties,
+saturated logits, out-of-bounds canaries and CUDA-graph replay.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_expert_routing_token_b200 as moe
+import oracle
+from moe_expert_routing_token_b200 import inputs
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def run_gpu(op, x, bias, k, renorm, G, TG, rsf):
+    xd = x.to(DEV)
+    if op == "softmax":
+        if G == 1 and TG == 1 and rsf == 1.0:
+            w, ids = moe.topk_softmax(xd, k, renorm)
+        else:
+            w, ids = moe.grouped_topk(xd, k, renorm, G, TG, rsf)
+    else:
+        bd = None if bias is None else bias.to(DEV)
+        w, ids = moe.biased_grouped_topk(xd, bd, k, renorm, G, TG, rsf)
+    torch.cuda.synchronize()
+    return w.cpu().numpy(), ids.cpu().numpy()
+
+
+def run_oracle(op, x, bias, k, renorm, G, TG, rsf):
+    if op == "softmax":
+        return oracle.grouped_topk(x, k, renorm, G, TG, rsf)
+    return oracle.biased_grouped_topk(x, bias, k, renorm, G, TG, rsf)
+
+
+def check(op, x, bias, k, renorm, G, TG, rsf):
+    w, ids = run_gpu(op, x, bias, k, renorm, G, TG, rsf)
+    orc = run_oracle(op, x, bias, k, renorm, G, TG, rsf)
+    rep = parity.compare(w, ids, orc, E=x.shape[1], G=G, TG=TG, k=k, renorm=renorm, rsf=rsf,
+                         fp32_logits=(x.dtype == torch.float32))
+    assert rep.ok(), rep.summary()
+    return rep
+
+
+def _spec_args(name):
+    sp = inputs.SPECS[name]
+    op = "softmax" if name in ("softmax", "grouped") else "sigmoid"
+    return op, sp.topk, sp.renormalize, sp.num_expert_group, sp.topk_group, sp.routed_scaling_factor
+
+
+@pytest.mark.parametrize("name,M", [(n, m) for n in ("softmax", "sigmoid", "biased", "grouped")
+                                    for m in inputs.SIZES[n]])
+def test_workloads_full_size(name, M):
+    d = inputs.make(name, M)
+    op, k, renorm, G, TG, rsf = _spec_args(name)
+    rep = check(op, d["logits"], d["bias"], k, renorm, G, TG, rsf)
+    # near ties must stay rare on these draws
+    assert rep.near_tie <= max(3, M // 200), rep.summary()
+
+
+@pytest.mark.parametrize("name", ["softmax", "sigmoid", "biased", "grouped"])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 17, 31, 33, 63, 129, 1000, 4099])
+def test_ragged_batches(name, M):
+    d = inputs.make(name, M, seed=77 + M)
+    op, k, renorm, G, TG, rsf = _spec_args(name)
+    check(op, d["logits"], d["bias"], k, renorm, G, TG, rsf)
+
+
+@pytest.mark.parametrize("name", ["softmax", "sigmoid", "biased", "grouped"])
+def test_other_dtype(name):
+    """bf16 for the fp32 workloads and fp32 for the bf16 ones."""
+    d = inputs.make(name, 777, seed=5)
+    x = d["logits"]
+    x = x.to(torch.bfloat16) if x.dtype == torch.float32 else x.to(torch.float32)
+    op, k, renorm, G, TG, rsf = _spec_args(name)
+    check(op, x, d["bias"], k, renorm, G, TG, rsf)
+
+
+# (op, E, G, TG, k, renorm, rsf, bias) across the three kernel families
+SHAPES = [
+    ("sigmoid", 256, 8, 4, 8, True, 2.5, True),    # segment, DeepSeek-V3
+    ("sigmoid", 256, 4, 2, 6, False, 1.0, True),   # segment, 2 lanes per group
+    ("sigmoid", 256, 2, 1, 7, True, 1.0, True),    # segment, odd k
+    ("sigmoid", 256, 1, 1, 1, True, 1.0, False),   # segment, no bias, k=1
+    ("sigmoid", 256, 8, 8, 32, True, 1.0, True),   # segment, k=32, all groups kept
+    ("softmax", 256, 8, 4, 8, True, 1.0, False),   # segment, softmax on 256
+    ("softmax", 160, 8, 3, 6, True, 2.0, False),   # segment, renormalised
+    ("softmax", 160, 1, 1, 4, False, 1.0, False),  # segment, E=160 ungrouped
+    ("sigmoid", 160, 8, 2, 4, True, 1.0, True),    # segment, sigmoid on 160
+    ("softmax", 8, 1, 1, 2, True, 1.0, False),     # small
+    ("softmax", 16, 4, 2, 3, False, 1.0, False),   # small, grouped
+    ("sigmoid", 32, 4, 2, 5, True, 1.5, True),     # small, biased
+    ("sigmoid", 8, 2, 1, 4, True, 1.0, True),      # small, k = admissible
+    ("softmax", 64, 8, 3, 5, True, 1.0, False),    # generic
+    ("sigmoid", 128, 16, 4, 8, True, 2.5, True),   # generic
+    ("sigmoid", 384, 8, 4, 8, True, 2.5, True),    # generic
+    ("softmax", 1024, 32, 8, 16, False, 1.0, False),  # generic, large
+    ("sigmoid", 256, 16, 4, 8, True, 2.5, True),   # generic (lanes would straddle groups)
+    ("sigmoid", 72, 9, 3, 6, True, 1.0, True),     # generic, odd group count
+]
+
+
+@pytest.mark.parametrize("op,E,G,TG,k,renorm,rsf,use_bias", SHAPES)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_kernel_families(op, E, G, TG, k, renorm, rsf, use_bias, dtype):
+    M = 531
+    x = inputs.random_logits(M, E, 2.0, dtype, seed=E * 31 + G * 7 + k)
+    bias = inputs.random_bias(E, 0.05, seed=E + 1) if use_bias else None
+    check(op, x, bias, k, renorm, G, TG, rsf)
+
+
+@pytest.mark.parametrize("op,E,G,TG,k", [("sigmoid", 256, 8, 4, 8), ("sigmoid", 256, 1, 1, 8),
+                                         ("softmax", 160, 8, 3, 6), ("softmax", 8, 1, 1, 2),
+                                         ("sigmoid", 64, 4, 2, 4)])
+def test_all_equal_logits_pick_lowest_indices(op, E, G, TG, k):
+    """Massive ties (exact-fallback path): the lowest indices win, exactly."""
+    x = torch.zeros(70, E, dtype=torch.bfloat16)
+    w, ids = run_gpu(op, x, None, k, True, G, TG, 1.0)
+    orc = run_oracle(op, x, None, k, True, G, TG, 1.0)
+    assert np.array_equal(ids, orc.ids)
+    assert np.allclose(w, 1.0 / k, rtol=1e-6)
+
+
+def test_some_rows_tied_some_not():
+    """A warp that mixes tied and clear rows takes the exact path for all."""
+    d = inputs.make("biased", 64, seed=3)
+    x = d["logits"].clone()
+    x[5] = 0
+    x[6, :64] = 1.0
+    op, k, renorm, G, TG, rsf = _spec_args("biased")
+    check(op, x, None, k, renorm, G, TG, rsf)
+
+
+@pytest.mark.parametrize("scale", [20.0, 60.0, 120.0])
+def test_saturated_logits(scale):
+    """Large logits saturate the sigmoid; ties among saturated scores are
+    near ties and must still be valid choices."""
+    x = inputs.random_logits(300, 256, scale, torch.float32, seed=int(scale))
+    bias = inputs.random_bias(256, 0.05, seed=9)
+    check("sigmoid", x, bias, 8, True, 8, 4, 2.5)
+    check("softmax", x, None, 8, True, 8, 4, 1.0)
+
+
+def test_outputs_have_no_out_of_bounds_writes():
+    M, k = 1000, 8
+    d = inputs.make("biased", M)
+    x = d["logits"].to(DEV)
+    b = d["bias"].to(DEV)
+    pad = 4096
+    wbuf = torch.full((M * k + 2 * pad,), 12345.0, device=DEV)
+    ibuf = torch.full((M * k + 2 * pad,), -777, dtype=torch.int32, device=DEV)
+    w = wbuf[pad:pad + M * k].view(M, k)
+    ids = ibuf[pad:pad + M * k].view(M, k)
+    moe.biased_grouped_topk(x, b, k, True, 8, 4, 2.5, out=(w, ids))
+    torch.cuda.synchronize()
+    assert torch.all(wbuf[:pad] == 12345.0) and torch.all(wbuf[pad + M * k:] == 12345.0)
+    assert torch.all(ibuf[:pad] == -777) and torch.all(ibuf[pad + M * k:] == -777)
+    assert torch.all((ids >= 0) & (ids < 256))
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_cuda_graph_replay_matches_eager(M):
+    d = inputs.make("sigmoid", M)
+    x = d["logits"].to(DEV)
+    b = d["bias"].to(DEV)
+    w0, i0 = moe.biased_grouped_topk(x, b, 8, True, 1, 1)
+    w = torch.empty_like(w0)
+    ids = torch.empty_like(i0)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        moe.biased_grouped_topk(x, b, 8, True, 1, 1, out=(w, ids))  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.biased_grouped_topk(x, b, 8, True, 1, 1, out=(w, ids))
+    w.zero_()
+    ids.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(ids, i0) and torch.equal(w, w0)
+
+
+def test_invalid_arguments_raise_before_launch():
+    x = torch.zeros(4, 256, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError):
+        moe.biased_grouped_topk(x, None, 8, True, 3, 1)      # 3 does not divide 256
+    with pytest.raises(ValueError):
+        moe.grouped_topk(x, 8, True, 8, 0)
+    with pytest.raises(NotImplementedError):
+        moe.topk_softmax(x, 33, True)
+
+
+def test_empty_batch():
+    x = torch.zeros(0, 256, dtype=torch.bfloat16, device=DEV)
+    w, ids = moe.biased_grouped_topk(x, None, 8, True, 8, 4)
+    assert w.shape == (0, 8) and ids.shape == (0, 8)
