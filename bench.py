@@ -285,7 +285,9 @@ def run_ours(args):
     M = args.M or DEFAULT_M[name]
     sp = inputs.SPECS[name]
     d = inputs.make(name, M, seed=inputs.default_seed(name, M) + 7919 * rank)
-    stream = torch.cuda.current_stream(dev)
+    # a dedicated stream: graphs cannot be captured on the legacy default stream
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
     sptr = stream.cuda_stream
 
     # ---- rotating device pool larger than L2 --------------------------------

@@ -90,6 +90,16 @@ MOE_API const char* moe_status_string(int status);
 MOE_API const char* moe_last_error(void);
 
 /*
+ * moe_watchdog_trips - number of times, since the library was loaded on the
+ * current device, that one of its kernels gave up on a barrier wait after the
+ * wait's time limit (about 2 s) instead of spinning for ever.  A kernel that
+ * trips the watchdog stops early and its outputs for that call are
+ * unspecified.  Zero in normal operation.  Synchronises with the device (it is
+ * a diagnostic, not for the hot path).  count: host pointer, out.
+ */
+MOE_API int moe_watchdog_trips(unsigned int* count);
+
+/*
  * moe_topk_softmax - [R] §2: softmax over each row, top-k, optional
  * renormalise (the sgl_kernel topk_softmax(topk_weights, topk_ids,
  * gating_output, renormalize) call).

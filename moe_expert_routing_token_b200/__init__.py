@@ -16,9 +16,10 @@ from .routing import (  # noqa: F401
     grouped_topk,
     lib,
     topk_softmax,
+    watchdog_trips,
 )
 
 __all__ = [
     "topk_softmax", "grouped_topk", "biased_grouped_topk", "fused_router_topk",
-    "fused_router_workspace_size", "lib", "RoutingError",
+    "fused_router_workspace_size", "lib", "RoutingError", "watchdog_trips",
 ]

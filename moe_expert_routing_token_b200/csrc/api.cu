@@ -17,6 +17,8 @@
 #include "fused_router.cuh"
 #include "moe_routing.h"
 #include "routing_kernels.cuh"
+#include "routing_staged.cuh"
+#include "tma_host.cuh"
 
 namespace moe {
 
@@ -106,16 +108,69 @@ int launch_rows(Kernel k, int threads, size_t smem, int64_t rows_per_block, cons
 
 bool aligned(const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
 
+// Experts per lane for E = 256 (32: 8 lanes per row; 16: 16 lanes per row).
+#ifndef MOE_SEG_C256
+#define MOE_SEG_C256 32
+#endif
+constexpr int kC256 = MOE_SEG_C256;
+
 template <typename TIn, int SCORE, bool BIAS>
 int launch_segment(int E, const RouteArgs& a, cudaStream_t st) {
     if (E == 256) {
-        constexpr int L = 256 / 32, R = 32 / L;
-        return launch_rows(route_segment_kernel<TIn, 256, 32, SCORE, BIAS>, kSegThreads, 0,
+        constexpr int L = 256 / kC256, R = 32 / L;
+        return launch_rows(route_segment_kernel<TIn, 256, kC256, SCORE, BIAS>, kSegThreads, 0,
                            (kSegThreads / 32) * R, a, st);
     }
     constexpr int L = 160 / 20, R = 32 / L;
     return launch_rows(route_segment_kernel<TIn, 160, 20, SCORE, BIAS>, kSegThreads, 0,
                        (kSegThreads / 32) * R, a, st);
+}
+
+// Batches at least this large take the TMA-staged streaming kernel.
+constexpr int64_t kStagedMinRows = 1024;
+
+template <typename TIn, int E, int C, int SCORE, bool BIAS>
+int launch_staged_ec(const RouteArgs& a, cudaStream_t st) {
+    using Cfg = StagedCfg<TIn, E, C, SCORE, BIAS>;
+    auto kern = route_staged_kernel<TIn, E, C, SCORE, BIAS>;
+    const int threads = (Cfg::W + 1) * 32;
+    int dev = 0, sms = 0, per_sm = 1;
+    int rc = device_and_sms(&dev, &sms);
+    if (rc != MOE_OK) return rc;
+    {
+        // raise the dynamic shared memory limit once per device
+        static std::mutex mu;
+        static bool done[64] = {};
+        std::lock_guard<std::mutex> lk(mu);
+        if (!done[dev & 63]) {
+            cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)Cfg::SMEM);
+            if (err != cudaSuccess) return cuda_fail(err, "cudaFuncSetAttribute(staged routing)");
+            done[dev & 63] = true;
+        }
+    }
+    rc = resident_blocks(dev, kern, threads, Cfg::SMEM, &per_sm);
+    if (rc != MOE_OK) return rc;
+    CUtensorMap tmap;
+    cudaError_t err = encode_tmap_2d(&tmap, a.logits,
+                                     sizeof(TIn) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                                     (uint64_t)a.M, (uint64_t)E, (uint64_t)E * sizeof(TIn), Cfg::BOX_E,
+                                     Cfg::RB, true);
+    if (err != cudaSuccess) return cuda_fail(err, "cuTensorMapEncodeTiled(logits)");
+    const int64_t nblocks = (a.M + Cfg::RB - 1) / Cfg::RB;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const int grid = (int)(nblocks < cap ? nblocks : cap);
+    kern<<<grid, threads, Cfg::SMEM, st>>>(tmap, a, nblocks);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail(err, "staged routing kernel launch");
+    return MOE_OK;
+}
+
+template <typename TIn, int SCORE, bool BIAS>
+int launch_staged(int E, const RouteArgs& a, cudaStream_t st) {
+    if (E == 256) return launch_staged_ec<TIn, 256, kC256, SCORE, BIAS>(a, st);
+    return launch_staged_ec<TIn, 160, 20, SCORE, BIAS>(a, st);
 }
 
 template <typename TIn, int SCORE, bool BIAS>
@@ -141,10 +196,12 @@ template <typename TIn, int SCORE, bool BIAS>
 int dispatch_typed(const RouteArgs& a, cudaStream_t st) {
     const int E = a.E;
     const size_t esz = sizeof(TIn);
-    if ((E == 256 || E == 160) && (E == 256 ? 8 : 8) % a.G == 0) {
-        const int C = (E == 256) ? 32 : 20;
+    if ((E == 256 || E == 160) && (E == 256 ? 256 / kC256 : 8) % a.G == 0) {
+        const int C = (E == 256) ? kC256 : 20;
         const size_t chunk = C * esz;
         const size_t vec = (chunk % 16 == 0) ? 16 : 8;
+        if (a.M >= kStagedMinRows && aligned(a.logits, 16) && (E * esz) % 16 == 0)
+            return launch_staged<TIn, SCORE, BIAS>(E, a, st);
         if (aligned(a.logits, vec)) return launch_segment<TIn, SCORE, BIAS>(E, a, st);
     }
     if ((E == 8 || E == 16 || E == 32) && aligned(a.logits, 16))
@@ -203,6 +260,14 @@ int route(const void* logits, int dtype, const float* bias, int64_t M, int E, in
 
 }  // namespace
 
+int read_routing_watchdog(unsigned int* count) {
+    unsigned int v = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(&v, g_watchdog_trips_routing, sizeof(v));
+    if (err != cudaSuccess) return cuda_fail(err, "cudaMemcpyFromSymbol(watchdog)");
+    *count = v;
+    return MOE_OK;
+}
+
 int set_error(int status, const char* msg) { return fail(status, "%s", msg); }
 int set_cuda_error(cudaError_t err, const char* what) { return cuda_fail(err, what); }
 int sm_count(int* dev, int* sms) { return device_and_sms(dev, sms); }
@@ -229,6 +294,17 @@ const char* moe_status_string(int status) {
 }
 
 const char* moe_last_error(void) { return moe::g_last_error; }
+
+int moe_watchdog_trips(unsigned int* count) {
+    if (!count) return moe::fail(MOE_ERR_INVALID_ARG, "moe_watchdog_trips: null pointer");
+    unsigned int a = 0, b = 0;
+    int rc = moe::read_routing_watchdog(&a);
+    if (rc != MOE_OK) return rc;
+    rc = moe::read_fused_watchdog(&b);
+    if (rc != MOE_OK) return rc;
+    *count = a + b;
+    return MOE_OK;
+}
 
 int moe_topk_softmax(const void* gating_output, int dtype, int64_t M, int32_t E, int32_t topk,
                      int32_t renormalize, float* topk_weights, int32_t* topk_ids, void* stream) {

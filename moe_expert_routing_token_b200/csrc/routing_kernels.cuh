@@ -36,86 +36,102 @@ constexpr int kCandCap = 32;
 
 __device__ __forceinline__ unsigned seg_bits(int L) { return L >= 32 ? kFullMask : ((1u << L) - 1u); }
 
-template <typename TIn, int E, int C, int SCORE, bool BIAS>
-__global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a) {
-    constexpr int L = E / C;   // lanes per row
-    constexpr int R = 32 / L;  // rows per warp
-    constexpr int WARPS = kSegThreads / 32;
-    constexpr int CQ = (C / 4) | 1;  // odd number of float4 per lane: conflict-free STS.128
-    constexpr int CS = CQ * 4;
-    constexpr int TPL = (32 + L - 1) / L;  // output ranks per lane (k <= 32)
+// Per-warp routing of R rows, L lanes per row, C consecutive experts per lane.
+// `xin` holds the lane's C logits (fp32); everything after the load - scoring,
+// group selection, candidate ranking, weights and the output stores - is here
+// so that the standalone routing kernel and the fused router's epilogue run
+// the same code.  `s_bias` is the correction bias in shared memory in the
+// padded lane-chunk layout written by load_bias_padded() (ignored without
+// BIAS): chunk j (experts [jC, jC+C)) starts at float j*CS, CS an odd number
+// of float4, so the 16-byte reads of the L lanes of a segment hit distinct
+// banks.
+template <int E, int C, int SCORE, bool BIAS>
+struct SegRouter {
+    static constexpr int L = E / C;   // lanes per row
+    static constexpr int R = 32 / L;  // rows per warp
+    static constexpr int CQ = (C / 4) | 1;  // odd number of float4 per lane: conflict-free STS.128
+    static constexpr int CS = CQ * 4;
+    static constexpr int TPL = (32 + L - 1) / L;  // output ranks per lane (k <= 32)
     static_assert(E % C == 0 && 32 % L == 0 && C % 4 == 0 && C <= 32, "bad segment shape");
 
-    __shared__ __align__(16) float s_p[WARPS][R * L * CS];  // unbiased score (softmax: logit)
-    __shared__ float2 s_cand[WARPS][R][kCandCap + 1];     // candidate (key, id)
-    __shared__ float s_candp[WARPS][R][kCandCap];         // candidate unbiased score
-    __shared__ float2 s_out[WARPS][R][32];                // by rank: (score, id)
-    __shared__ float s_bias[BIAS ? E : 1];
+    static constexpr int BIAS_FLOATS = L * CS;  // padded bias layout
 
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int seg = lane / L;
-    const int sl = lane % L;
-    const int base = seg * L;
-    const int e0 = sl * C;
+    struct Scratch {                            // one per warp; rows padded against bank conflicts
+        unsigned long long cand[R][kCandCap + 1];  // candidate order keys
+        float candp[R][kCandCap + 1];           // candidate unbiased score
+        float2 out[R][33];                      // by rank: (score, id)
+    };
 
-    float b_r[C];
-    if constexpr (BIAS) {
-        for (int e = threadIdx.x; e < E; e += blockDim.x) s_bias[e] = __ldg(a.bias + e);
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < C; ++i) b_r[i] = s_bias[e0 + i];
+    // Copy the (E,) bias from global memory into the padded layout; called
+    // by every thread of the block, followed by a barrier.
+    __device__ __forceinline__ static void load_bias_padded(const float* g_bias, float* s_bias) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) s_bias[(e / C) * CS + e % C] = __ldg(g_bias + e);
     }
 
-    const int G = a.G, TG = a.TG, K = a.K;
-    const int P = L / G;  // lanes per group (the dispatcher guarantees G | L)
-    const int g = sl / P;
-    const bool all_groups = (TG == G);
-    const int nsel_lanes = all_groups ? L : TG * P;
-    const int need = (K + 1) >> 1;
-    const unsigned smask = seg_bits(L) << base;
-
-    float* my_p = &s_p[warp][(seg * L + sl) * CS];
-    const TIn* logits = static_cast<const TIn*>(a.logits);
-    const int64_t step = (int64_t)gridDim.x * WARPS * R;
-
-    for (int64_t row0 = ((int64_t)blockIdx.x * WARPS + warp) * R; row0 < a.M; row0 += step) {
-        const int64_t row = row0 + seg;
-        const bool valid = row < a.M;
-
-        float x[C];
-        if (valid) {
-            ChunkLoader<TIn, C>::load(logits + row * E + e0, x);
-        } else {
-#pragma unroll
-            for (int i = 0; i < C; ++i) x[i] = 0.0f;
+    // Unbiased scores kept in a per-warp shared buffer (for callers whose raw
+    // logits are not in shared memory).
+    struct StoredScores {
+        float* warp_p;  // R * L * CS floats
+        __device__ __forceinline__ void store(int q, float p0, float p1, float p2, float p3) const {
+            const int lane = threadIdx.x & 31;
+            reinterpret_cast<float4*>(warp_p + (lane / L * L + lane % L) * CS)[q] = make_float4(p0, p1, p2, p3);
         }
+        __device__ __forceinline__ float get(int seg, int e) const {
+            return warp_p[(seg * L + e / C) * CS + e % C];
+        }
+    };
+
+    template <class PSrc>
+    __device__ __forceinline__ static void route(const float (&xin)[C], bool valid, int64_t row,
+                                                 const float* s_bias, Scratch& sc, const RouteArgs& a,
+                                                 const PSrc& psrc) {
+        const int lane = threadIdx.x & 31;
+        const int seg = lane / L;
+        const int sl = lane % L;
+        const int base = seg * L;
+        const int e0 = sl * C;
+        const int G = a.G, TG = a.TG, K = a.K;
+        const int P = L / G;  // lanes per group (the dispatcher guarantees G | L)
+        const int g = sl / P;
+        const bool all_groups = (TG == G);
+        const int nsel_lanes = all_groups ? L : TG * P;
+        const int need = (K + 1) >> 1;
+        const unsigned smask = seg_bits(L) << base;
 
         // Pass 1: score, selection key, per-lane top-2 of the keys.
         float key[C];
-        float m1 = -INFINITY, m2 = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            const float p = (SCORE == kSigmoid) ? sigmoid_f32(x[i]) : x[i];
-            x[i] = p;
-            key[i] = BIAS ? p + b_r[i] : p;
-            top2_push(m1, m2, key[i]);
+        for (int q = 0; q < C / 4; ++q) {
+            float pv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                pv[j] = (SCORE == kSigmoid) ? sigmoid_f32(xin[4 * q + j]) : xin[4 * q + j];
+            psrc.store(q, pv[0], pv[1], pv[2], pv[3]);
+            if constexpr (BIAS) {
+                const float4 b = reinterpret_cast<const float4*>(s_bias + sl * CS)[q];
+                key[4 * q + 0] = pv[0] + b.x;
+                key[4 * q + 1] = pv[1] + b.y;
+                key[4 * q + 2] = pv[2] + b.z;
+                key[4 * q + 3] = pv[3] + b.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) key[4 * q + j] = pv[j];
+            }
         }
-#pragma unroll
-        for (int q = 0; q < C / 4; ++q)
-            reinterpret_cast<float4*>(my_p)[q] =
-                make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+        float m1, m2;
+        top2_of(key, m1, m2);
 
-        // Group score from the group's lanes, then keep the TG best groups.
-        float g1 = m1, g2 = m2;
-        for (int o = 1; o < P; o <<= 1) {
-            const float b1 = __shfl_xor_sync(kFullMask, g1, o);
-            const float b2 = __shfl_xor_sync(kFullMask, g2, o);
-            top2_merge(g1, g2, b1, b2);
-        }
-        const float gs = (a.group_kind == kGroupTop2Sum) ? g1 + g2 : g1;
+        // Group score from the group's lanes, then keep the TG best groups
+        // (nothing to do when every group is kept).
         bool gsel = true;
         if (!all_groups) {
+            float g1 = m1, g2 = m2;
+            for (int o = 1; o < P; o <<= 1) {
+                const float b1 = __shfl_xor_sync(kFullMask, g1, o);
+                const float b2 = __shfl_xor_sync(kFullMask, g2, o);
+                top2_merge(g1, g2, b1, b2);
+            }
+            const float gs = (a.group_kind == kGroupTop2Sum) ? g1 + g2 : g1;
             int rank = 0;
             for (int h = 0; h < G; ++h) {
                 const float o = __shfl_sync(kFullMask, gs, base + h * P);
@@ -150,12 +166,19 @@ __global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a)
         unsigned mask = 0u;
         if (gsel) {
 #pragma unroll
-            for (int i = 0; i < C; ++i) mask |= (key[i] >= tau ? 1u : 0u) << i;
+            for (int i = 0; i < C; ++i)
+                if (key[i] >= tau) mask |= 1u << i;
         }
+        // Inclusive prefix of the per-lane counts over the segment; its last
+        // lane holds the segment total n.
         const int cnt = __popc(mask);
-        int n = cnt;
+        int incl = cnt;
 #pragma unroll
-        for (int o = L / 2; o >= 1; o >>= 1) n += __shfl_xor_sync(kFullMask, n, o);
+        for (int o = 1; o < L; o <<= 1) {
+            const int t = __shfl_up_sync(kFullMask, incl, o);
+            if (sl >= o) incl += t;
+        }
+        const int n = __shfl_sync(kFullMask, incl, base + L - 1);
 
         const bool exact_needed = valid && (n > kCandCap || n < K);
         if (__any_sync(kFullMask, exact_needed)) {
@@ -186,42 +209,40 @@ __global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a)
                 if (bi >= 0 && wi == e0 + bi) taken |= 1u << bi;
                 if (sl == 0) {
                     const int gi = (wi >= 0 && wi < E) ? wi : 0;
-                    s_out[warp][seg][j] =
-                        make_float2(s_p[warp][(seg * L + gi / C) * CS + gi % C], __int_as_float(gi));
+                    sc.out[seg][j] = make_float2(psrc.get(seg, gi), __int_as_float(gi));
                 }
             }
             __syncwarp();
         } else {
             // Compact the candidates of the segment into shared memory ...
-            int incl = cnt;
-#pragma unroll
-            for (int o = 1; o < L; o <<= 1) {
-                const int t = __shfl_up_sync(kFullMask, incl, o);
-                if (sl >= o) incl += t;
-            }
             int pos = incl - cnt;
             unsigned mm = valid ? mask : 0u;
             while (mm) {
                 const int b = __ffs(mm) - 1;
                 mm &= mm - 1u;
-                const float pv = my_p[b];
-                const float kv = BIAS ? pv + s_bias[e0 + b] : pv;
-                s_cand[warp][seg][pos] = make_float2(kv, __int_as_float(e0 + b));
-                s_candp[warp][seg][pos] = pv;
+                const float pv = psrc.get(seg, e0 + b);
+                const float kv = BIAS ? pv + s_bias[sl * CS + b] : pv;
+                sc.cand[seg][pos] = order_key(kv, e0 + b);
+                sc.candp[seg][pos] = pv;
                 ++pos;
             }
             __syncwarp();
-            // ... and rank each one by counting the candidates that beat it.
+            // ... and rank each one by counting the candidates that beat it
+            // (a lane takes candidates sl and sl + L in one pass).
             const int nn = valid ? n : 0;
-            for (int t = sl; t < nn; t += L) {
-                const float2 c = s_cand[warp][seg][t];
-                const int ci = __float_as_int(c.y);
-                int r = 0;
+            for (int t = sl; t < nn; t += 2 * L) {
+                const int t2 = t + L;
+                const unsigned long long c0 = sc.cand[seg][t];
+                const unsigned long long c1 = t2 < nn ? sc.cand[seg][t2] : ~0ull;
+                int r0 = 0, r1 = 0;
                 for (int u = 0; u < nn; ++u) {
-                    const float2 d = s_cand[warp][seg][u];
-                    r += beats(d.x, __float_as_int(d.y), c.x, ci) ? 1 : 0;
+                    const unsigned long long d = sc.cand[seg][u];
+                    r0 += d > c0 ? 1 : 0;
+                    r1 += d > c1 ? 1 : 0;
                 }
-                if (r < K) s_out[warp][seg][r] = make_float2(s_candp[warp][seg][t], c.y);
+                if (r0 < K) sc.out[seg][r0] = make_float2(sc.candp[seg][t], __int_as_float(order_key_index(c0)));
+                if (t2 < nn && r1 < K)
+                    sc.out[seg][r1] = make_float2(sc.candp[seg][t2], __int_as_float(order_key_index(c1)));
             }
             __syncwarp();
         }
@@ -251,7 +272,7 @@ __global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a)
             w_loc[q] = 0.0f;
             id_loc[q] = 0;
             if (t < K) {
-                const float2 o = s_out[warp][seg][t];
+                const float2 o = sc.out[seg][t];
                 const float w = (SCORE == kSoftmax) ? exp_f32(o.x - rowmax) : o.x;
                 w_loc[q] = w;
                 id_loc[q] = __float_as_int(o.y);
@@ -262,9 +283,9 @@ __global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a)
         if (a.renorm) {
 #pragma unroll
             for (int o = L / 2; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
-            scale = a.rsf / sum;
+            scale = __fdiv_rn(a.rsf, sum);
         } else {
-            scale = (SCORE == kSoftmax) ? a.rsf / denom_all : a.rsf;
+            scale = (SCORE == kSoftmax) ? __fdiv_rn(a.rsf, denom_all) : a.rsf;
         }
         if (valid) {
 #pragma unroll
@@ -277,6 +298,44 @@ __global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a)
             }
         }
         __syncwarp();
+    }
+};
+
+template <typename TIn, int E, int C, int SCORE, bool BIAS>
+__global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a) {
+    using Router = SegRouter<E, C, SCORE, BIAS>;
+    constexpr int L = Router::L;
+    constexpr int R = Router::R;
+    constexpr int WARPS = kSegThreads / 32;
+
+    __shared__ __align__(16) typename Router::Scratch s_scratch[WARPS];
+    __shared__ __align__(16) float s_p[WARPS][R * L * Router::CS];
+    __shared__ __align__(16) float s_bias[BIAS ? Router::BIAS_FLOATS : 4];
+
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int seg = lane / L;
+    const int e0 = (lane % L) * C;
+
+    if constexpr (BIAS) {
+        Router::load_bias_padded(a.bias, s_bias);
+        __syncthreads();
+    }
+
+    const TIn* logits = static_cast<const TIn*>(a.logits);
+    const int64_t step = (int64_t)gridDim.x * WARPS * R;
+    for (int64_t row0 = ((int64_t)blockIdx.x * WARPS + warp) * R; row0 < a.M; row0 += step) {
+        const int64_t row = row0 + seg;
+        const bool valid = row < a.M;
+        float x[C];
+        if (valid) {
+            ChunkLoader<TIn, C>::load(logits + row * E + e0, x);
+        } else {
+#pragma unroll
+            for (int i = 0; i < C; ++i) x[i] = 0.0f;
+        }
+        Router::route(x, valid, row, s_bias, s_scratch[warp], a,
+                      typename Router::StoredScores{s_p[warp]});
     }
 }
 

@@ -35,6 +35,7 @@ SIGNATURES = {
     "moe_abi_version": (ctypes.c_int, []),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_error": (ctypes.c_char_p, []),
+    "moe_watchdog_trips": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint)]),
     "moe_topk_softmax": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_grouped_topk": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _i32, _i32, _i32, _i32, _f32,
                                         _vp, _vp, _vp]),
@@ -161,6 +162,13 @@ def biased_grouped_topk(gating_output: torch.Tensor, correction_bias, topk: int,
                                        _stream(gating_output.device))
     _check(st, "moe_biased_grouped_topk")
     return w, ids
+
+
+def watchdog_trips() -> int:
+    """Times a library kernel gave up on a barrier wait (0 in normal use)."""
+    n = ctypes.c_uint(0)
+    _check(lib().moe_watchdog_trips(ctypes.byref(n)), "moe_watchdog_trips")
+    return n.value
 
 
 def fused_router_workspace_size(M: int, K: int, E: int) -> int:

@@ -73,9 +73,11 @@ def test_ragged_batches(name, M):
 
 
 @pytest.mark.parametrize("name", ["softmax", "sigmoid", "biased", "grouped"])
-def test_other_dtype(name):
-    """bf16 for the fp32 workloads and fp32 for the bf16 ones."""
-    d = inputs.make(name, 777, seed=5)
+@pytest.mark.parametrize("M", [777, 2777])
+def test_other_dtype(name, M):
+    """bf16 for the fp32 workloads and fp32 for the bf16 ones (direct-load and
+    TMA-staged paths)."""
+    d = inputs.make(name, M, seed=5)
     x = d["logits"]
     x = x.to(torch.bfloat16) if x.dtype == torch.float32 else x.to(torch.float32)
     op, k, renorm, G, TG, rsf = _spec_args(name)
@@ -108,8 +110,8 @@ SHAPES = [
 
 @pytest.mark.parametrize("op,E,G,TG,k,renorm,rsf,use_bias", SHAPES)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_kernel_families(op, E, G, TG, k, renorm, rsf, use_bias, dtype):
-    M = 531
+@pytest.mark.parametrize("M", [531, 1500])
+def test_kernel_families(op, E, G, TG, k, renorm, rsf, use_bias, dtype, M):
     x = inputs.random_logits(M, E, 2.0, dtype, seed=E * 31 + G * 7 + k)
     bias = inputs.random_bias(E, 0.05, seed=E + 1) if use_bias else None
     check(op, x, bias, k, renorm, G, TG, rsf)
@@ -201,3 +203,9 @@ def test_empty_batch():
     x = torch.zeros(0, 256, dtype=torch.bfloat16, device=DEV)
     w, ids = moe.biased_grouped_topk(x, None, 8, True, 8, 4)
     assert w.shape == (0, 8) and ids.shape == (0, 8)
+
+
+def test_no_watchdog_trips():
+    """No kernel gave up on a barrier wait during the tests above."""
+    torch.cuda.synchronize()
+    assert moe.watchdog_trips() == 0
