@@ -1,13 +1,422 @@
-// Fused router: hidden_states x router_weight on the tensor cores, routing on
-// the fp32 accumulator (SGLang MoE routing page, §5 Fused MoE Router).
+// Fused router: logits = hidden_states x router_weight on the tcgen05 tensor
+// cores, then the biased grouped top-k routing on the fp32 accumulator
+// (SGLang MoE routing page, §5 Fused MoE Router: the router projection and the
+// top-k selection in one kernel, logits never stored; §4 for the routing).
+//
+// Design (one 128-token tile per cluster of SPLIT CTAs, one CTA per SM):
+//   warp 0      TMA producer: A = hidden tile (128 x 64, K-major) and B = the
+//               router weight tile (64 x 256) into a 4-stage ring, 128-byte
+//               swizzle; B is K-major for (E, K) weights and MN-major for
+//               (K, E) weights.
+//   warp 1      allocates 256 TMEM columns and issues tcgen05.mma
+//               (kind::f16, M=128, N=256, K=16, bf16 in, fp32 accumulate)
+//               from one lane; tcgen05.commit frees a stage when its MMAs
+//               are done and signals the epilogue after the last one.
+//   warps 2..5  epilogue: the split-K partial sums are exchanged through
+//               distributed shared memory (each CTA of the cluster owns
+//               128/SPLIT rows and receives the other CTAs' partials for
+//               them), summed in a fixed rank order, staged in shared memory
+//               and routed by the same SegRouter body as the routing kernels.
+// The K dimension is split across the SPLIT CTAs of a cluster so that enough
+// SMs stream the hidden states (M=8192: 64 tiles x 2 = 128 CTAs; decode
+// M=64: 1 tile x 16).  Every barrier wait is bounded.
+#include <cstdio>
+#include <mutex>
+#include <type_traits>
+
 #include "fused_router.cuh"
 #include "moe_routing.h"
+#include "routing_kernels.cuh"
+#include "sm100_ptx.cuh"
+#include "tma_host.cuh"
 
 namespace moe {
-int read_fused_watchdog(unsigned int* count) {
-    *count = 0;
-    return 0;
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;
+constexpr int kBBytes = kBN * kBK * 2;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
+constexpr int kRecvStride = 260;        // floats per received partial row (bank spread)
+constexpr int kFinStride = 8 * 36 + 4;  // floats per staged logits row: 8 chunks of 36
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+using Router = SegRouter<256, 32, kSigmoid, true>;
+using RouterNB = SegRouter<256, 32, kSigmoid, false>;
+
+static __device__ unsigned int g_watchdog_trips_fused;
+
+struct FusedArgs {
+    RouteArgs route;   // M, E, G, TG, K (topk), group_kind, renorm, rsf, bias, outputs
+    float* logits_out; // (M, 256) fp32 or nullptr
+    int num_kb;        // K / 64
+    int kb_per_split;
+};
+
+__host__ __device__ constexpr size_t fused_smem_bytes() {
+    return 1024 + (size_t)kStages * kStageBytes + Router::BIAS_FLOATS * 4 + 256;
 }
+
+// Owner-side staged logits row: chunk c (32 floats) at c * 36.
+__device__ __forceinline__ int fin_off(int r, int col) { return r * kFinStride + (col >> 5) * 36 + (col & 31); }
+
+template <int SPLIT>
+struct FinScores {
+    const float* fin;
+    int warp_row0;
+    __device__ __forceinline__ void store(int, float, float, float, float) const {}
+    __device__ __forceinline__ float get(int seg, int e) const {
+        const int r = warp_row0 + seg;  // rows past the owned range are padding
+        return r < kBM / SPLIT ? sigmoid_f32(fin[fin_off(r, e)]) : 0.0f;
+    }
+};
+
+template <int SPLIT, bool B_MN_MAJOR, bool BIAS>
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_router_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        FusedArgs fa) {
+    using R_t = typename std::conditional<BIAS, Router, RouterNB>::type;
+    constexpr int ROWS = kBM / SPLIT;  // rows of the tile this CTA routes
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* s_bias = reinterpret_cast<float*>(smem + (size_t)kStages * kStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(s_bias + Router::BIAS_FLOATS);
+    uint64_t* empty = full + kStages;
+    uint64_t* accum = empty + kStages;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    volatile int* s_peer_abort = s_abort + 1;
+    // Overlays of the stage ring, valid once the main loop is over.
+    float* recv = reinterpret_cast<float*>(smem);                                   // [SPLIT-1][ROWS][260]
+    float* fin = recv + (size_t)(SPLIT - 1) * ROWS * kRecvStride;                   // [ROWS][292]
+    auto* scratch = reinterpret_cast<typename R_t::Scratch*>(fin + (size_t)ROWS * kFinStride);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const int m_tile = blockIdx.x / SPLIT;
+    const int kb0 = (int)rank * fa.kb_per_split;
+    int nkb = fa.num_kb - kb0;
+    if (nkb > fa.kb_per_split) nkb = fa.kb_per_split;
+    if (nkb < 0) nkb = 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        ptx::mbar_init(accum, 1);
+        *s_abort = 0;
+        *s_peer_abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if constexpr (BIAS) Router::load_bias_padded(fa.route.bias, s_bias);
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_holder, 256);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0 && nkb > 0) {
+            ptx::tma_prefetch_desc(&tmA);
+            ptx::tma_prefetch_desc(&tmB);
+            const uint64_t pol_a = ptx::l2_policy_evict_first();
+            const uint64_t pol_b = ptx::l2_policy_evict_last();
+            int kb = 0;
+            for (; kb < nkb; ++kb) {
+                const int s = kb % kStages;
+                if (!ptx::mbar_wait(&empty[s], ((kb / kStages) & 1) ^ 1, kWaitNs)) {
+                    *s_abort = 1;
+                    atomicAdd(&g_watchdog_trips_fused, 1u);
+                    break;
+                }
+                uint8_t* a_s = smem + (size_t)s * kStageBytes;
+                uint8_t* b_s = a_s + kABytes;
+                const int kc = (kb0 + kb) * kBK;
+                ptx::mbar_arrive_expect_tx(&full[s], kStageBytes);
+                ptx::tma_load_2d(a_s, &tmA, kc, m_tile * kBM, &full[s], pol_a);
+                if constexpr (B_MN_MAJOR) {
+#pragma unroll
+                    for (int j = 0; j < kBN / 64; ++j)
+                        ptx::tma_load_2d(b_s + j * 8192, &tmB, j * 64, kc, &full[s], pol_b);
+                } else {
+                    ptx::tma_load_2d(b_s, &tmB, kc, 0, &full[s], pol_b);
+                }
+            }
+            // Leave only once the copies issued have landed (bounded).
+            for (int k = 0; k < kStages && k < kb; ++k) {
+                const int j = kb - 1 - k;
+                ptx::mbar_wait(&full[j % kStages], (j / kStages) & 1, kWaitNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN, B_MN_MAJOR);
+            for (int kb = 0; kb < nkb && !*s_abort; ++kb) {
+                const int s = kb % kStages;
+                if (!ptx::mbar_wait(&full[s], (kb / kStages) & 1, kWaitNs)) {
+                    *s_abort = 1;
+                    atomicAdd(&g_watchdog_trips_fused, 1u);
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t a_addr = ptx::smem_u32(smem + (size_t)s * kStageBytes);
+                const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    const uint64_t adesc = ptx::sdesc_sw128(a_addr + kk * 32, 16, 1024);
+                    const uint64_t bdesc = B_MN_MAJOR ? ptx::sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                                      : ptx::sdesc_sw128(b_addr + kk * 32, 16, 1024);
+                    ptx::umma_bf16(tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                }
+                ptx::umma_commit(&empty[s]);
+            }
+            ptx::umma_commit(accum);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue: wait for the accumulator
+        if (!ptx::mbar_wait(accum, 0, kWaitNs)) {
+            if (lane == 0) atomicAdd(&g_watchdog_trips_fused, 1u);
+            *s_abort = 1;
+        }
+        ptx::tc_fence_after();
+    }
+    __syncwarp();
+
+    // All MMAs of this CTA are complete (the epilogue waited on `accum`), so
+    // the stage ring can be reused as the receive buffer.
+    ptx::cluster_sync();
+
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;            // tile row of this thread's TMEM lane
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const bool epi = warp >= 2;
+    const bool has_acc = nkb > 0;           // uniform over the CTA
+    const int owner = r / ROWS;
+    // tcgen05.ld is warp-collective (.sync.aligned): whole warps load, lanes
+    // only predicate what they do with the values.
+    const bool warp_sends = epi && !(q * 32 >= (int)rank * ROWS && q * 32 + 32 <= ((int)rank + 1) * ROWS);
+    const bool warp_owns = epi && (q * 32 < ((int)rank + 1) * ROWS) && (q * 32 + 32 > (int)rank * ROWS);
+    if (warp_sends) {
+        // Send the partial sums of rows owned by other CTAs to their owners.
+        const bool sends = owner != (int)rank;
+        const int slot = (int)rank < owner ? (int)rank : (int)rank - 1;
+        const uint32_t dst = ptx::map_to_rank(
+            ptx::smem_u32(recv + ((size_t)slot * ROWS + (r - owner * ROWS)) * kRecvStride), sends ? owner : rank);
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+            float v[32];
+            __syncwarp();
+            if (has_acc) {
+                ptx::tmem_ld32(t_row + c * 32, v);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+            }
+            if (sends) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    ptx::st_cluster_f32x4(dst + (c * 32 + 4 * i) * 4, v[4 * i], v[4 * i + 1], v[4 * i + 2],
+                                          v[4 * i + 3]);
+            }
+        }
+        if (sends && *s_abort)
+            ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(const_cast<int*>(s_peer_abort)), owner), 1u);
+    }
+    ptx::cluster_sync();
+
+    // Owners: sum the partials in rank order and stage the logits.
+    const int64_t row_base = (int64_t)m_tile * kBM + (int64_t)rank * ROWS;
+    if (warp_owns) {
+        const bool owns = owner == (int)rank;
+        const int lr = owns ? r - owner * ROWS : 0;
+        const int64_t grow = row_base + lr;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+            float own[32];
+            __syncwarp();
+            if (has_acc) {
+                ptx::tmem_ld32(t_row + c * 32, own);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) own[i] = 0.0f;
+            }
+            if (!owns) continue;
+            float acc[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+            for (int src = 0; src < SPLIT; ++src) {
+                if (src == (int)rank) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] += own[i];
+                } else {
+                    const int slot = src < (int)rank ? src : src - 1;
+                    const float4* p = reinterpret_cast<const float4*>(
+                        recv + ((size_t)slot * ROWS + lr) * kRecvStride + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 t = p[i];
+                        acc[4 * i] += t.x;
+                        acc[4 * i + 1] += t.y;
+                        acc[4 * i + 2] += t.z;
+                        acc[4 * i + 3] += t.w;
+                    }
+                }
+            }
+            float4* f = reinterpret_cast<float4*>(fin + fin_off(lr, c * 32));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+            if (fa.logits_out != nullptr && grow < fa.route.M) {
+                float4* g = reinterpret_cast<float4*>(fa.logits_out + grow * kBN + c * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    g[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 256);
+    }
+
+    // Routing of the owned rows by the four epilogue warps (4 rows each).
+    if (epi) {
+        const bool aborted = *s_abort || *s_peer_abort;
+        const int ew = warp - 2;
+        const int seg = lane / R_t::L;
+        const int e0 = (lane % R_t::L) * 32;
+        for (int base = 0; base < ROWS; base += kEpiWarps * R_t::R) {
+            const int warp_row0 = base + ew * R_t::R;
+            const int lr = warp_row0 + seg;
+            const int64_t grow = row_base + lr;
+            const bool valid = lr < ROWS && grow < fa.route.M;
+            float x[32];
+            if (lr < ROWS) {
+                const float4* p = reinterpret_cast<const float4*>(fin + fin_off(lr, e0));
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 t = p[i];
+                    x[4 * i] = t.x;
+                    x[4 * i + 1] = t.y;
+                    x[4 * i + 2] = t.z;
+                    x[4 * i + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+            }
+            R_t::route(x, valid, grow, s_bias, scratch[ew], fa.route, FinScores<SPLIT>{fin, warp_row0});
+            if (aborted && valid && (lane % R_t::L) == 0) {
+                for (int t = 0; t < fa.route.K; ++t) fa.route.ids[grow * fa.route.K + t] = -1;
+            }
+        }
+    }
+}
+
+template <int SPLIT, bool B_MN, bool BIAS>
+int launch_fused(const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs& fa, int m_tiles,
+                 cudaStream_t stream) {
+    auto kern = fused_router_kernel<SPLIT, B_MN, BIAS>;
+    {
+        static std::mutex mu;
+        static bool done[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        std::lock_guard<std::mutex> lk(mu);
+        if (!done[dev & 63]) {
+            cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)fused_smem_bytes());
+            if (err != cudaSuccess) return set_cuda_error(err, "cudaFuncSetAttribute(fused router smem)");
+            if (SPLIT > 8) {
+                err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+                if (err != cudaSuccess) return set_cuda_error(err, "cudaFuncSetAttribute(cluster size)");
+            }
+            done[dev & 63] = true;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(m_tiles * SPLIT), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = fused_smem_bytes();
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = SPLIT;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, fa);
+    if (err != cudaSuccess) return set_cuda_error(err, "fused router launch");
+    return MOE_OK;
+}
+
+template <bool B_MN, bool BIAS>
+int launch_split(int split, const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs& fa,
+                 int m_tiles, cudaStream_t st) {
+    switch (split) {
+        case 2: return launch_fused<2, B_MN, BIAS>(tmA, tmB, fa, m_tiles, st);
+        case 4: return launch_fused<4, B_MN, BIAS>(tmA, tmB, fa, m_tiles, st);
+        case 8: return launch_fused<8, B_MN, BIAS>(tmA, tmB, fa, m_tiles, st);
+        default: return launch_fused<16, B_MN, BIAS>(tmA, tmB, fa, m_tiles, st);
+    }
+}
+
+// Largest split whose cluster of one-CTA-per-SM blocks can be scheduled.
+int max_schedulable_split(int dev) {
+    static std::mutex mu;
+    static int cached[64] = {};
+    std::lock_guard<std::mutex> lk(mu);
+    if (cached[dev & 63]) return cached[dev & 63];
+    int best = 8;
+    auto kern = fused_router_kernel<16, false, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem_bytes()) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(16, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = fused_smem_bytes();
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 16;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) best = 16;
+    }
+    cudaGetLastError();
+    cached[dev & 63] = best;
+    return best;
+}
+
+}  // namespace
+
+int read_fused_watchdog(unsigned int* count) {
+    unsigned int v = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(&v, g_watchdog_trips_fused, sizeof(v));
+    if (err != cudaSuccess) return set_cuda_error(err, "cudaMemcpyFromSymbol(fused watchdog)");
+    *count = v;
+    return MOE_OK;
+}
+
 }  // namespace moe
 
 extern "C" {
@@ -23,11 +432,102 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
                           int32_t topk_group, float routed_scaling_factor, float* topk_weights,
                           int32_t* topk_ids, float* logits_out, void* workspace,
                           size_t workspace_bytes, void* stream) {
-    (void)hidden_states; (void)router_weight; (void)weight_layout; (void)correction_bias;
-    (void)M; (void)K; (void)E; (void)topk; (void)renormalize; (void)num_expert_group;
-    (void)topk_group; (void)routed_scaling_factor; (void)topk_weights; (void)topk_ids;
-    (void)logits_out; (void)workspace; (void)workspace_bytes; (void)stream;
-    return moe::set_error(MOE_ERR_UNSUPPORTED, "moe_fused_router_topk: not built yet");
+    (void)workspace;
+    (void)workspace_bytes;
+    using namespace moe;
+    const char* who = "moe_fused_router_topk";
+    char msg[256];
+    if (M < 0) {
+        snprintf(msg, sizeof msg, "%s: M=%lld < 0", who, (long long)M);
+        return set_error(MOE_ERR_INVALID_ARG, msg);
+    }
+    if (K < 1 || E < 1) {
+        snprintf(msg, sizeof msg, "%s: K=%d and E=%d must be positive", who, K, E);
+        return set_error(MOE_ERR_INVALID_ARG, msg);
+    }
+    if (weight_layout != MOE_WEIGHT_K_BY_E && weight_layout != MOE_WEIGHT_E_BY_K) {
+        snprintf(msg, sizeof msg, "%s: weight_layout %d is not MOE_WEIGHT_K_BY_E or MOE_WEIGHT_E_BY_K", who,
+                 weight_layout);
+        return set_error(MOE_ERR_INVALID_ARG, msg);
+    }
+    if (num_expert_group < 1 || E % num_expert_group != 0 || topk_group < 1 || topk_group > num_expert_group ||
+        topk < 1 || topk > topk_group * (E / num_expert_group) || !(routed_scaling_factor == routed_scaling_factor) ||
+        routed_scaling_factor > 3.4e38f || routed_scaling_factor < -3.4e38f) {
+        snprintf(msg, sizeof msg, "%s: invalid routing arguments (E=%d G=%d TG=%d topk=%d)", who, E,
+                 num_expert_group, topk_group, topk);
+        return set_error(MOE_ERR_INVALID_ARG, msg);
+    }
+    if (E != 256) {
+        snprintf(msg, sizeof msg, "%s: E=%d; this build supports E=256", who, E);
+        return set_error(MOE_ERR_UNSUPPORTED, msg);
+    }
+    if (K % 64 != 0) {
+        snprintf(msg, sizeof msg, "%s: K=%d is not a multiple of 64", who, K);
+        return set_error(MOE_ERR_UNSUPPORTED, msg);
+    }
+    if (8 % num_expert_group != 0 || topk > 32) {
+        snprintf(msg, sizeof msg, "%s: num_expert_group=%d / topk=%d not supported", who, num_expert_group, topk);
+        return set_error(MOE_ERR_UNSUPPORTED, msg);
+    }
+    if (M == 0) return MOE_OK;
+    if (!hidden_states || !router_weight || !topk_weights || !topk_ids)
+        return set_error(MOE_ERR_INVALID_ARG, "moe_fused_router_topk: null pointer argument");
+    auto al = [](const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; };
+    if (!al(hidden_states, 16) || !al(router_weight, 16) || (logits_out && !al(logits_out, 16)) ||
+        !al(topk_weights, 4) || !al(topk_ids, 4) || (correction_bias && !al(correction_bias, 4)))
+        return set_error(MOE_ERR_INVALID_ARG,
+                         "moe_fused_router_topk: hidden_states/router_weight/logits_out must be 16-byte "
+                         "aligned, outputs and bias 4-byte aligned");
+
+    int dev = 0, sms = 0;
+    int rc = sm_count(&dev, &sms);
+    if (rc != MOE_OK) return rc;
+
+    CUtensorMap tmA, tmB;
+    cudaError_t err = encode_tmap_2d(&tmA, hidden_states, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)M,
+                                     (uint64_t)K, (uint64_t)K * 2, kBK, kBM, true);
+    if (err != cudaSuccess) return set_cuda_error(err, "cuTensorMapEncodeTiled(hidden_states)");
+    const bool b_mn = weight_layout == MOE_WEIGHT_K_BY_E;
+    if (b_mn)
+        err = encode_tmap_2d(&tmB, router_weight, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)K, (uint64_t)E,
+                             (uint64_t)E * 2, 64, kBK, true);
+    else
+        err = encode_tmap_2d(&tmB, router_weight, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)E, (uint64_t)K,
+                             (uint64_t)K * 2, kBK, kBN, true);
+    if (err != cudaSuccess) return set_cuda_error(err, "cuTensorMapEncodeTiled(router_weight)");
+
+    const int m_tiles = (int)((M + kBM - 1) / kBM);
+    const int num_kb = K / kBK;
+    int split = 2;
+    const int per = sms / (m_tiles > 0 ? m_tiles : 1);
+    if (per >= 16) split = 16;
+    else if (per >= 8) split = 8;
+    else if (per >= 4) split = 4;
+    if (split == 16 && max_schedulable_split(dev) < 16) split = 8;
+    while (split > 2 && split > num_kb) split >>= 1;
+
+    FusedArgs fa;
+    fa.route.logits = nullptr;
+    fa.route.bias = correction_bias;
+    fa.route.M = M;
+    fa.route.E = E;
+    fa.route.G = num_expert_group;
+    fa.route.TG = topk_group;
+    fa.route.K = topk;
+    fa.route.group_kind = kGroupTop2Sum;
+    fa.route.renorm = renormalize ? 1 : 0;
+    fa.route.rsf = routed_scaling_factor;
+    fa.route.weights = topk_weights;
+    fa.route.ids = topk_ids;
+    fa.logits_out = logits_out;
+    fa.num_kb = num_kb;
+    fa.kb_per_split = (num_kb + split - 1) / split;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (b_mn)
+        return correction_bias ? launch_split<true, true>(split, tmA, tmB, fa, m_tiles, st)
+                               : launch_split<true, false>(split, tmA, tmB, fa, m_tiles, st);
+    return correction_bias ? launch_split<false, true>(split, tmA, tmB, fa, m_tiles, st)
+                           : launch_split<false, false>(split, tmA, tmB, fa, m_tiles, st);
 }
 
 }  // extern "C"
