@@ -12,7 +12,7 @@
 //               (kind::f16, M=128, N=256, K=16, bf16 in, fp32 accumulate)
 //               from one lane; tcgen05.commit frees a stage when its MMAs
 //               are done and signals the epilogue after the last one.
-//   warps 2..5  epilogue: the split-K partial sums are exchanged through
+//   warps 2..9  epilogue: the split-K partial sums are exchanged through
 //               distributed shared memory (each CTA of the cluster owns
 //               128/SPLIT rows and receives the other CTAs' partials for
 //               them), summed in a fixed rank order, staged in shared memory
@@ -41,10 +41,10 @@ constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kBBytes = kBN * kBK * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4;
-constexpr int kRecvStride = 260;        // floats per received partial row (bank spread)
-constexpr int kFinStride = 8 * 36 + 4;  // floats per staged logits row: 8 chunks of 36
+constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kFinStride = 8 * 36 + 4;  // floats per staged row: 8 chunks of 36 (bank spread)
+constexpr int kPrefetchAhead = 6;       // k-blocks of A brought into L2 ahead of their load
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 using Router = SegRouter<256, 32, kSigmoid, true>;
@@ -93,10 +93,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* s_peer_abort = s_abort + 1;
-    // Overlays of the stage ring, valid once the main loop is over.
-    float* recv = reinterpret_cast<float*>(smem);                                   // [SPLIT-1][ROWS][260]
-    float* fin = recv + (size_t)(SPLIT - 1) * ROWS * kRecvStride;                   // [ROWS][292]
-    auto* scratch = reinterpret_cast<typename R_t::Scratch*>(fin + (size_t)ROWS * kFinStride);
+    // Overlays of the stage ring, valid once the main loop is over: one slot
+    // of partial sums per source CTA for the rows this CTA owns, in the
+    // chunked staged-row layout; slot 0 is summed in place and then holds
+    // the logits that are routed.
+    float* slots = reinterpret_cast<float*>(smem);                                // [SPLIT][ROWS][292]
+    float* fin = slots;
+    // Router scratch reuses slots 1.. once they have been summed into slot 0.
+    auto* scratch = reinterpret_cast<typename R_t::Scratch*>(slots + (size_t)ROWS * kFinStride);
+    static_assert((size_t)(SPLIT - 1) * ROWS * kFinStride * 4 >= kEpiWarps * sizeof(typename R_t::Scratch),
+                  "router scratch must fit in the summed slots");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -107,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (nkb > fa.kb_per_split) nkb = fa.kb_per_split;
     if (nkb < 0) nkb = 0;
 
+    ptx::griddep_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(&full[s], 1);
@@ -116,12 +123,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         *s_abort = 0;
         *s_peer_abort = 0;
         ptx::fence_mbar_init();
+        ptx::tma_prefetch_desc(&tmA);
+        ptx::tma_prefetch_desc(&tmB);
     }
-    if constexpr (BIAS) Router::load_bias_padded(fa.route.bias, s_bias);
     if (warp == 1) {
         ptx::tmem_alloc(tmem_holder, 256);
         ptx::tmem_relinquish();
     }
+    // The prologue above overlaps the previous kernel; inputs are read after it.
+    ptx::griddep_wait();
+    if constexpr (BIAS) Router::load_bias_padded(fa.route.bias, s_bias);
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -130,8 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         if (lane == 0 && nkb > 0) {
-            ptx::tma_prefetch_desc(&tmA);
-            ptx::tma_prefetch_desc(&tmB);
             const uint64_t pol_a = ptx::l2_policy_evict_first();
             const uint64_t pol_b = ptx::l2_policy_evict_last();
             int kb = 0;
@@ -145,6 +154,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t* a_s = smem + (size_t)s * kStageBytes;
                 uint8_t* b_s = a_s + kABytes;
                 const int kc = (kb0 + kb) * kBK;
+                if (kb == 0) {
+                    for (int j = 1; j <= kPrefetchAhead && j < nkb; ++j)
+                        ptx::tma_prefetch_l2_2d(&tmA, (kb0 + j) * kBK, m_tile * kBM);
+                } else if (kb + kPrefetchAhead < nkb) {
+                    ptx::tma_prefetch_l2_2d(&tmA, (kb0 + kb + kPrefetchAhead) * kBK, m_tile * kBM);
+                }
                 ptx::mbar_arrive_expect_tx(&full[s], kStageBytes);
                 ptx::tma_load_2d(a_s, &tmA, kc, m_tile * kBM, &full[s], pol_a);
                 if constexpr (B_MN_MAJOR) {
@@ -200,24 +215,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the stage ring can be reused as the receive buffer.
     ptx::cluster_sync();
 
-    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int q = warp & 3;                 // TMEM lane quarter of this warp (warps 2..9 -> 2,3,0,1,2,3,0,1)
     const int r = q * 32 + lane;            // tile row of this thread's TMEM lane
     const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const bool epi = warp >= 2;
     const bool has_acc = nkb > 0;           // uniform over the CTA
-    const int owner = r / ROWS;
-    // tcgen05.ld is warp-collective (.sync.aligned): whole warps load, lanes
-    // only predicate what they do with the values.
-    const bool warp_sends = epi && !(q * 32 >= (int)rank * ROWS && q * 32 + 32 <= ((int)rank + 1) * ROWS);
-    const bool warp_owns = epi && (q * 32 < ((int)rank + 1) * ROWS) && (q * 32 + 32 > (int)rank * ROWS);
-    if (warp_sends) {
-        // Send the partial sums of rows owned by other CTAs to their owners.
-        const bool sends = owner != (int)rank;
-        const int slot = (int)rank < owner ? (int)rank : (int)rank - 1;
+    if (epi) {
+        // Every tile row's partial sums go to slot `rank` of the CTA that
+        // owns the row (this CTA included).  tcgen05.ld is warp-collective:
+        // whole warps load, lanes only choose the destination.
+        const int owner = r / ROWS;
         const uint32_t dst = ptx::map_to_rank(
-            ptx::smem_u32(recv + ((size_t)slot * ROWS + (r - owner * ROWS)) * kRecvStride), sends ? owner : rank);
+            ptx::smem_u32(slots + ((size_t)rank * ROWS + (r - owner * ROWS)) * kFinStride), owner);
+        const int half = (warp - 2) >> 2;  // which half of the columns this warp moves
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = half * (kBN / 64); c < (half + 1) * (kBN / 64); ++c) {
             float v[32];
             __syncwarp();
             if (has_acc) {
@@ -226,65 +238,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.0f;
             }
-            if (sends) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    ptx::st_cluster_f32x4(dst + (c * 32 + 4 * i) * 4, v[4 * i], v[4 * i + 1], v[4 * i + 2],
-                                          v[4 * i + 3]);
-            }
+            for (int i = 0; i < 8; ++i)
+                ptx::st_cluster_f32x4(dst + (c * 36 + 4 * i) * 4, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
-        if (sends && *s_abort)
+        if (*s_abort && half == 0)
             ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(const_cast<int*>(s_peer_abort)), owner), 1u);
     }
     ptx::cluster_sync();
 
-    // Owners: sum the partials in rank order and stage the logits.
+    // Sum the SPLIT partials of the owned rows in rank order, all 128
+    // epilogue threads in parallel, in place into slot 0.
     const int64_t row_base = (int64_t)m_tile * kBM + (int64_t)rank * ROWS;
-    if (warp_owns) {
-        const bool owns = owner == (int)rank;
-        const int lr = owns ? r - owner * ROWS : 0;
+    if (epi) {
+        constexpr int COLS = kBN * ROWS / (kEpiWarps * 32);  // columns per thread
+        const int t = threadIdx.x - 64;
+        const int lr = t % ROWS;
+        const int col0 = (t / ROWS) * COLS;
         const int64_t grow = row_base + lr;
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-            float own[32];
-            __syncwarp();
-            if (has_acc) {
-                ptx::tmem_ld32(t_row + c * 32, own);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) own[i] = 0.0f;
+        for (int col = col0; col < col0 + COLS; col += 4) {
+            const int off = lr * kFinStride + (col >> 5) * 36 + (col & 31);
+            float4 acc = *reinterpret_cast<const float4*>(slots + off);
+            for (int src = 1; src < SPLIT; ++src) {
+                const float4 v = *reinterpret_cast<const float4*>(slots + (size_t)src * ROWS * kFinStride + off);
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
             }
-            if (!owns) continue;
-            float acc[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-            for (int src = 0; src < SPLIT; ++src) {
-                if (src == (int)rank) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[i] += own[i];
-                } else {
-                    const int slot = src < (int)rank ? src : src - 1;
-                    const float4* p = reinterpret_cast<const float4*>(
-                        recv + ((size_t)slot * ROWS + lr) * kRecvStride + c * 32);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 t = p[i];
-                        acc[4 * i] += t.x;
-                        acc[4 * i + 1] += t.y;
-                        acc[4 * i + 2] += t.z;
-                        acc[4 * i + 3] += t.w;
-                    }
-                }
-            }
-            float4* f = reinterpret_cast<float4*>(fin + fin_off(lr, c * 32));
-#pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-            if (fa.logits_out != nullptr && grow < fa.route.M) {
-                float4* g = reinterpret_cast<float4*>(fa.logits_out + grow * kBN + c * 32);
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    g[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-            }
+            *reinterpret_cast<float4*>(slots + off) = acc;
+            if (fa.logits_out != nullptr && grow < fa.route.M)
+                *reinterpret_cast<float4*>(fa.logits_out + grow * kBN + col) = acc;
         }
     }
     ptx::tc_fence_before();
@@ -354,13 +339,15 @@ int launch_fused(const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = fused_smem_bytes();
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = SPLIT;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t err = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, fa);
     if (err != cudaSuccess) return set_cuda_error(err, "fused router launch");
     return MOE_OK;

@@ -48,6 +48,49 @@ __device__ __forceinline__ float sigmoid_f32(float x) {
     return r;
 }
 
+// Packed fp32 pairs (sm_100 paired FADD/FMUL).
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+    return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float lo2(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi2(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// Smallest logit the pair sigmoid accepts: 1 + 2^(43.5 log2 e) stays below
+// 2^63, so the product of two denominators cannot overflow.  sigmoid(-43.5)
+// is 1.3e-19; clamping lower logits to it moves a score by less than that.
+constexpr float kSigmoidClamp = -43.5f;
+constexpr uint32_t kSigmoidClampBf16x2 = 0xC22EC22Eu;  // bf16 -43.5 in both halves
+
+// Logistic function of two values with one reciprocal:
+// 1/d0 = d1 * rcp(d0 d1), 1/d1 = d0 * rcp(d0 d1), d = 1 + 2^(-x log2 e).
+// Inputs must be >= kSigmoidClamp.  Relative error ~3e-7; used for the
+// selection keys (the weights use sigmoid_f32 on the raw logit).
+__device__ __forceinline__ unsigned long long sigmoid_pair(unsigned long long x) {
+    const unsigned long long t = mul2(x, pack2(-1.4426950408889634f, -1.4426950408889634f));
+    float e0, e1, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(lo2(t)));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(hi2(t)));
+    const unsigned long long d = add2(pack2(e0, e1), pack2(1.0f, 1.0f));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(lo2(d) * hi2(d)));
+    return mul2(pack2(hi2(d), lo2(d)), pack2(r, r));
+}
+
+__device__ __forceinline__ uint32_t clamp_bf16x2_for_sigmoid(uint32_t w) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(kSigmoidClampBf16x2));
+    return r;
+}
+
 // e^x for the softmax: 2^(x * log2(e)) with the hardware approximation.
 __device__ __forceinline__ float exp_f32(float x) {
     float e;
@@ -110,6 +153,63 @@ __device__ __forceinline__ void top2_of(const float (&v)[N], float& m1, float& m
     }
     m1 = h[0];
     m2 = l[0];
+}
+
+// Compare-exchange for descending order.
+__device__ __forceinline__ void cx_desc(float& a, float& b) {
+    const float hi = fmaxf(a, b);
+    b = fminf(a, b);
+    a = hi;
+}
+
+// Sort a bitonic sequence of N (power of two) values into descending order.
+template <int N>
+__device__ __forceinline__ void bitonic_clean_desc(float (&x)[N]) {
+#pragma unroll
+    for (int k = N / 2; k >= 1; k >>= 1) {
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            if ((i & k) == 0) cx_desc(x[i], x[i + k]);
+    }
+}
+
+// Over the aligned segment of L lanes, each lane contributing its sorted
+// pair (v1 >= v2), return in every lane the 8 largest of the 2L values,
+// descending (padded with -inf when 2L < 8).  Log2(L) xor-shuffle steps, each
+// merging two sorted lists with a bitonic network.
+template <int L>
+__device__ __forceinline__ void segment_top8(float v1, float v2, float (&out)[8]) {
+    float a[8] = {v1, v2, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    if constexpr (L >= 2) {  // two sorted pairs -> sorted 4
+        const float b0 = __shfl_xor_sync(kFullMask, a[0], 1);
+        const float b1 = __shfl_xor_sync(kFullMask, a[1], 1);
+        float y[4] = {a[0], a[1], b1, b0};
+        bitonic_clean_desc(y);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = y[i];
+    }
+    if constexpr (L >= 4) {  // two sorted 4-lists -> sorted 8
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[i] = a[i];
+            x[7 - i] = __shfl_xor_sync(kFullMask, a[i], 2);
+        }
+        bitonic_clean_desc(x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = x[i];
+    }
+#pragma unroll
+    for (int o = 4; o < L; o <<= 1) {  // two sorted 8-lists -> top 8
+        float b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) b[i] = __shfl_xor_sync(kFullMask, a[i], o);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], b[7 - i]);
+        bitonic_clean_desc(a);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = a[i];
 }
 
 template <typename T>

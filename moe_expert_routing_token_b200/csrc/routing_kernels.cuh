@@ -28,11 +28,13 @@
 #pragma once
 
 #include "routing_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 
 constexpr int kSegThreads = 128;
 constexpr int kCandCap = 32;
+constexpr int kCandStride = kCandCap + 4;  // room for sentinels to a multiple of 4; 16-B rows
 
 __device__ __forceinline__ unsigned seg_bits(int L) { return L >= 32 ? kFullMask : ((1u << L) - 1u); }
 
@@ -57,9 +59,23 @@ struct SegRouter {
     static constexpr int BIAS_FLOATS = L * CS;  // padded bias layout
 
     struct Scratch {                            // one per warp; rows padded against bank conflicts
-        unsigned long long cand[R][kCandCap + 1];  // candidate order keys
-        float candp[R][kCandCap + 1];           // candidate unbiased score
-        float2 out[R][33];                      // by rank: (score, id)
+        float keys[R * L * CS];                 // selection keys of pass 1 (lane-chunk layout)
+        unsigned long long cand[R][kCandStride];  // candidate order keys (+ zero sentinels)
+        float2 out[R][33];                      // by rank: (unbiased score, id)
+    };
+
+    // Raw logits kept in a per-warp shared buffer (for callers whose logits
+    // are not in shared memory); get() returns the unbiased score.
+    struct StoredScores {
+        float* warp_x;  // R * L * CS floats
+        __device__ __forceinline__ void store(int q, float x0, float x1, float x2, float x3) const {
+            const int lane = threadIdx.x & 31;
+            reinterpret_cast<float4*>(warp_x + (lane / L * L + lane % L) * CS)[q] = make_float4(x0, x1, x2, x3);
+        }
+        __device__ __forceinline__ float get(int seg, int e) const {
+            const float x = warp_x[(seg * L + e / C) * CS + e % C];
+            return SCORE == kSigmoid ? sigmoid_f32(x) : x;
+        }
     };
 
     // Copy the (E,) bias from global memory into the padded layout; called
@@ -70,18 +86,8 @@ struct SegRouter {
 
     // Unbiased scores kept in a per-warp shared buffer (for callers whose raw
     // logits are not in shared memory).
-    struct StoredScores {
-        float* warp_p;  // R * L * CS floats
-        __device__ __forceinline__ void store(int q, float p0, float p1, float p2, float p3) const {
-            const int lane = threadIdx.x & 31;
-            reinterpret_cast<float4*>(warp_p + (lane / L * L + lane % L) * CS)[q] = make_float4(p0, p1, p2, p3);
-        }
-        __device__ __forceinline__ float get(int seg, int e) const {
-            return warp_p[(seg * L + e / C) * CS + e % C];
-        }
-    };
-
-    template <class PSrc>
+    // XCLAMPED: the caller already raised sigmoid inputs to kSigmoidClamp.
+    template <bool XCLAMPED = false, class PSrc>
     __device__ __forceinline__ static void route(const float (&xin)[C], bool valid, int64_t row,
                                                  const float* s_bias, Scratch& sc, const RouteArgs& a,
                                                  const PSrc& psrc) {
@@ -97,26 +103,40 @@ struct SegRouter {
         const int nsel_lanes = all_groups ? L : TG * P;
         const int need = (K + 1) >> 1;
         const unsigned smask = seg_bits(L) << base;
+        float* my_keys = &sc.keys[(seg * L + sl) * CS];
 
         // Pass 1: score, selection key, per-lane top-2 of the keys.
         float key[C];
 #pragma unroll
         for (int q = 0; q < C / 4; ++q) {
-            float pv[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                pv[j] = (SCORE == kSigmoid) ? sigmoid_f32(xin[4 * q + j]) : xin[4 * q + j];
-            psrc.store(q, pv[0], pv[1], pv[2], pv[3]);
-            if constexpr (BIAS) {
-                const float4 b = reinterpret_cast<const float4*>(s_bias + sl * CS)[q];
-                key[4 * q + 0] = pv[0] + b.x;
-                key[4 * q + 1] = pv[1] + b.y;
-                key[4 * q + 2] = pv[2] + b.z;
-                key[4 * q + 3] = pv[3] + b.w;
+            psrc.store(q, xin[4 * q], xin[4 * q + 1], xin[4 * q + 2], xin[4 * q + 3]);
+            float4 b = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if constexpr (BIAS) b = reinterpret_cast<const float4*>(s_bias + sl * CS)[q];
+            unsigned long long k01, k23;
+            if constexpr (SCORE == kSigmoid) {
+                float x0 = xin[4 * q], x1 = xin[4 * q + 1], x2 = xin[4 * q + 2], x3 = xin[4 * q + 3];
+                if constexpr (!XCLAMPED) {
+                    x0 = fmaxf(x0, kSigmoidClamp);
+                    x1 = fmaxf(x1, kSigmoidClamp);
+                    x2 = fmaxf(x2, kSigmoidClamp);
+                    x3 = fmaxf(x3, kSigmoidClamp);
+                }
+                k01 = sigmoid_pair(pack2(x0, x1));
+                k23 = sigmoid_pair(pack2(x2, x3));
             } else {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) key[4 * q + j] = pv[j];
+                k01 = pack2(xin[4 * q], xin[4 * q + 1]);
+                k23 = pack2(xin[4 * q + 2], xin[4 * q + 3]);
             }
+            if constexpr (BIAS) {
+                k01 = add2(k01, pack2(b.x, b.y));
+                k23 = add2(k23, pack2(b.z, b.w));
+            }
+            key[4 * q + 0] = lo2(k01);
+            key[4 * q + 1] = hi2(k01);
+            key[4 * q + 2] = lo2(k23);
+            key[4 * q + 3] = hi2(k23);
+            reinterpret_cast<float4*>(my_keys)[q] =
+                make_float4(key[4 * q], key[4 * q + 1], key[4 * q + 2], key[4 * q + 3]);
         }
         float m1, m2;
         top2_of(key, m1, m2);
@@ -150,6 +170,15 @@ struct SegRouter {
 #pragma unroll
             for (int o = L / 2; o >= 1; o >>= 1) v = fminf(v, __shfl_xor_sync(kFullMask, v, o));
             tau = v;
+        } else if (K <= 8) {
+            // Tighter: the K-th largest of all kept lanes' top-2 values (those
+            // are K distinct kept experts).
+            float top[8];
+            segment_top8<L>(gsel ? m1 : -INFINITY, gsel ? m2 : -INFINITY, top);
+            tau = top[0];
+#pragma unroll
+            for (int i = 1; i < 8; ++i)
+                if (i == K - 1) tau = top[i];
         } else {
             const float my = gsel ? m2 : -INFINITY;
             int r = 0;
@@ -220,29 +249,36 @@ struct SegRouter {
             while (mm) {
                 const int b = __ffs(mm) - 1;
                 mm &= mm - 1u;
-                const float pv = psrc.get(seg, e0 + b);
-                const float kv = BIAS ? pv + s_bias[sl * CS + b] : pv;
-                sc.cand[seg][pos] = order_key(kv, e0 + b);
-                sc.candp[seg][pos] = pv;
+                sc.cand[seg][pos] = order_key(my_keys[b], e0 + b);
                 ++pos;
             }
+            // zero keys pad the list to a multiple of 4 (they beat nothing)
+            const int nn = valid ? n : 0;
+            const int n4 = (nn + 3) & ~3;
+            if (sl == 0)
+                for (int u = nn; u < n4; ++u) sc.cand[seg][u] = 0ull;
             __syncwarp();
             // ... and rank each one by counting the candidates that beat it
             // (a lane takes candidates sl and sl + L in one pass).
-            const int nn = valid ? n : 0;
             for (int t = sl; t < nn; t += 2 * L) {
                 const int t2 = t + L;
                 const unsigned long long c0 = sc.cand[seg][t];
                 const unsigned long long c1 = t2 < nn ? sc.cand[seg][t2] : ~0ull;
                 int r0 = 0, r1 = 0;
-                for (int u = 0; u < nn; ++u) {
-                    const unsigned long long d = sc.cand[seg][u];
-                    r0 += d > c0 ? 1 : 0;
-                    r1 += d > c1 ? 1 : 0;
+                for (int u = 0; u < n4; u += 4) {
+                    const ulonglong2 d01 = *reinterpret_cast<const ulonglong2*>(&sc.cand[seg][u]);
+                    const ulonglong2 d23 = *reinterpret_cast<const ulonglong2*>(&sc.cand[seg][u + 2]);
+                    r0 += (d01.x > c0) + (d01.y > c0) + (d23.x > c0) + (d23.y > c0);
+                    r1 += (d01.x > c1) + (d01.y > c1) + (d23.x > c1) + (d23.y > c1);
                 }
-                if (r0 < K) sc.out[seg][r0] = make_float2(sc.candp[seg][t], __int_as_float(order_key_index(c0)));
-                if (t2 < nn && r1 < K)
-                    sc.out[seg][r1] = make_float2(sc.candp[seg][t2], __int_as_float(order_key_index(c1)));
+                if (r0 < K) {
+                    const int id = order_key_index(c0);
+                    sc.out[seg][r0] = make_float2(psrc.get(seg, id), __int_as_float(id));
+                }
+                if (t2 < nn && r1 < K) {
+                    const int id = order_key_index(c1);
+                    sc.out[seg][r1] = make_float2(psrc.get(seg, id), __int_as_float(id));
+                }
             }
             __syncwarp();
         }
@@ -283,9 +319,9 @@ struct SegRouter {
         if (a.renorm) {
 #pragma unroll
             for (int o = L / 2; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
-            scale = __fdiv_rn(a.rsf, sum);
+            scale = __fdividef(a.rsf, sum);
         } else {
-            scale = (SCORE == kSoftmax) ? __fdiv_rn(a.rsf, denom_all) : a.rsf;
+            scale = (SCORE == kSoftmax) ? __fdividef(a.rsf, denom_all) : a.rsf;
         }
         if (valid) {
 #pragma unroll
@@ -317,6 +353,8 @@ __global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a)
     const int seg = lane / L;
     const int e0 = (lane % L) * C;
 
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     if constexpr (BIAS) {
         Router::load_bias_padded(a.bias, s_bias);
         __syncthreads();

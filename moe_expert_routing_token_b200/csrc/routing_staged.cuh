@@ -33,7 +33,12 @@ struct StagedCfg {
     static constexpr int CB = (E * ESZ + 127) / 128;      // 128-byte column blocks
     static constexpr int BOX_E = 128 / ESZ;               // elements per box row
     static constexpr int STAGE_BYTES = CB * RB * 128;
-    static constexpr int S = STAGE_BYTES <= 16384 ? 4 : 3;
+    // Stages: as many as fit (up to 4) while two blocks share an SM
+    // (<= ~113 KB each); a layout that cannot keep 2 stages that way runs
+    // one block per SM with 4 stages.
+    static constexpr int FIXED = 1024 + W * (int)sizeof(typename Router::Scratch) + Router::BIAS_FLOATS * 4 + 128;
+    static constexpr int S2 = (113 * 1024 - FIXED) / STAGE_BYTES;
+    static constexpr int S = S2 >= 2 ? (S2 > 4 ? 4 : S2) : 4;
     static constexpr int VEC = (C * ESZ) % 16 == 0 ? 16 : 8;  // bytes per chunk load
     static constexpr int BIAS_FLOATS = Router::BIAS_FLOATS;
     static constexpr size_t SMEM = 1024 + (size_t)S * STAGE_BYTES + W * sizeof(typename Router::Scratch) +
@@ -89,6 +94,7 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    ptx::griddep_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(&full[s], 1);
@@ -96,14 +102,17 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32)
         }
         *s_abort = 0;
         ptx::fence_mbar_init();
+        ptx::tma_prefetch_desc(&tmap);
     }
+    // Everything above overlaps the previous kernel in the stream; global
+    // inputs are read only after it has finished.
+    ptx::griddep_wait();
     if constexpr (BIAS) Router::load_bias_padded(a.bias, s_bias);
     __syncthreads();
 
     if (warp == W) {
         // ---------------- producer: one elected lane issues the TMA loads
         if (lane == 0) {
-            ptx::tma_prefetch_desc(&tmap);
             const uint64_t policy = ptx::l2_policy_evict_first();
             int it = 0;
             for (int64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x, ++it) {
@@ -151,7 +160,13 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32)
         if constexpr (Cfg::VEC == 16) {
 #pragma unroll
             for (int q = 0; q < C * Cfg::ESZ / 16; ++q) {
-                const uint4 v = *reinterpret_cast<const uint4*>(staged_addr<RB>(stage, r, e0 * Cfg::ESZ + 16 * q));
+                uint4 v = *reinterpret_cast<const uint4*>(staged_addr<RB>(stage, r, e0 * Cfg::ESZ + 16 * q));
+                if constexpr (sizeof(TIn) == 2 && SCORE == kSigmoid) {
+                    v.x = clamp_bf16x2_for_sigmoid(v.x);
+                    v.y = clamp_bf16x2_for_sigmoid(v.y);
+                    v.z = clamp_bf16x2_for_sigmoid(v.z);
+                    v.w = clamp_bf16x2_for_sigmoid(v.w);
+                }
                 if constexpr (sizeof(TIn) == 2) {
                     x[8 * q + 0] = bf16_lo(v.x); x[8 * q + 1] = bf16_hi(v.x);
                     x[8 * q + 2] = bf16_lo(v.y); x[8 * q + 3] = bf16_hi(v.y);
@@ -165,7 +180,11 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32)
         } else {
 #pragma unroll
             for (int q = 0; q < C * Cfg::ESZ / 8; ++q) {
-                const uint2 v = *reinterpret_cast<const uint2*>(staged_addr<RB>(stage, r, e0 * Cfg::ESZ + 8 * q));
+                uint2 v = *reinterpret_cast<const uint2*>(staged_addr<RB>(stage, r, e0 * Cfg::ESZ + 8 * q));
+                if constexpr (sizeof(TIn) == 2 && SCORE == kSigmoid) {
+                    v.x = clamp_bf16x2_for_sigmoid(v.x);
+                    v.y = clamp_bf16x2_for_sigmoid(v.y);
+                }
                 if constexpr (sizeof(TIn) == 2) {
                     x[4 * q + 0] = bf16_lo(v.x); x[4 * q + 1] = bf16_hi(v.x);
                     x[4 * q + 2] = bf16_lo(v.y); x[4 * q + 3] = bf16_hi(v.y);
@@ -174,8 +193,8 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32)
                 }
             }
         }
-        Router::route(x, valid, row, s_bias, scratch[warp], a,
-                      StagedScores<TIn, E, C, SCORE, BIAS>{stage, warp_row0});
+        Router::template route<sizeof(TIn) == 2>(x, valid, row, s_bias, scratch[warp], a,
+                                                 StagedScores<TIn, E, C, SCORE, BIAS>{stage, warp_row0});
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&empty[s]);
     }
