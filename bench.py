@@ -304,7 +304,7 @@ def run_ours(args):
     ws = [torch.empty(M, sp.topk, dtype=torch.float32, device=dev) for _ in range(pool)]
     ids = [torch.empty(M, sp.topk, dtype=torch.int32, device=dev) for _ in range(pool)]
     wsp_bytes = routing.fused_router_workspace_size(M, sp.K, sp.E) if name == "fused" else 0
-    wsp = [torch.empty(max(1, wsp_bytes), dtype=torch.uint8, device=dev) for _ in range(pool)]
+    wsp = [torch.zeros(max(1, wsp_bytes), dtype=torch.uint8, device=dev) for _ in range(pool)]
 
     dcode = routing.MOE_DTYPE_BF16 if sp.dtype == torch.bfloat16 else routing.MOE_DTYPE_F32
 
@@ -443,7 +443,7 @@ def e2e_measure(name, M, sp, d, dev, stream, world, args):
     hw = torch.empty(M, sp.topk, dtype=torch.float32).pin_memory()
     hi = torch.empty(M, sp.topk, dtype=torch.int32).pin_memory()
     need = routing.fused_router_workspace_size(M, sp.K, sp.E) if name == "fused" else 0
-    wsp = torch.empty(max(1, need), dtype=torch.uint8, device=dev)
+    wsp = torch.zeros(max(1, need), dtype=torch.uint8, device=dev)
 
     def step():
         x.copy_(src, non_blocking=True)

@@ -156,7 +156,10 @@ MOE_API int moe_biased_grouped_topk(const void* gating_output, int dtype,
 
 /*
  * moe_fused_router_workspace_size - bytes of device workspace that
- * moe_fused_router_topk needs for these sizes (0 when it needs none).
+ * moe_fused_router_topk needs for these sizes (0 when it needs none).  Small
+ * batches (M <= 128) with a long hidden size spread K over several
+ * thread-block clusters whose fp32 partial sums meet in the workspace
+ * ((clusters x M x 256) floats plus 256 bytes of arrival counters).
  * Returns (size_t)-1 for arguments moe_fused_router_topk would reject.
  */
 MOE_API size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E);
@@ -177,9 +180,11 @@ MOE_API size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E);
  *                   the routing consumed)
  *   workspace       device scratch of at least
  *                   moe_fused_router_workspace_size(M, K, E) bytes, 256-byte
- *                   aligned (NULL allowed when that size is 0).  Its contents
- *                   need no initialisation and are left in a state that the
- *                   next call accepts; calls that overlap on the GPU must not
+ *                   aligned (NULL allowed when that size is 0; otherwise a
+ *                   missing or short workspace is MOE_ERR_INVALID_ARG).  It
+ *                   must be zero-filled before its first use (its arrival
+ *                   counters start at zero); every call leaves it in that
+ *                   state again.  Calls that may overlap on the GPU must not
  *                   share one workspace.
  *   other arguments as moe_biased_grouped_topk
  */

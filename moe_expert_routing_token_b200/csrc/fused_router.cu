@@ -12,7 +12,7 @@
 //               (kind::f16, M=128, N=256, K=16, bf16 in, fp32 accumulate)
 //               from one lane; tcgen05.commit frees a stage when its MMAs
 //               are done and signals the epilogue after the last one.
-//   warps 2..9  epilogue: the split-K partial sums are exchanged through
+//   warps 2..17 epilogue: the split-K partial sums are exchanged through
 //               distributed shared memory (each CTA of the cluster owns
 //               128/SPLIT rows and receives the other CTAs' partials for
 //               them), summed in a fixed rank order, staged in shared memory
@@ -41,7 +41,7 @@ constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kBBytes = kBN * kBK * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter
+constexpr int kEpiWarps = 16;                // four per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kFinStride = 8 * 36 + 4;  // floats per staged row: 8 chunks of 36 (bank spread)
 constexpr int kPrefetchAhead = 6;       // k-blocks of A brought into L2 ahead of their load
@@ -53,11 +53,29 @@ using RouterNB = SegRouter<256, 32, kSigmoid, false>;
 static __device__ unsigned int g_watchdog_trips_fused;
 
 struct FusedArgs {
-    RouteArgs route;   // M, E, G, TG, K (topk), group_kind, renorm, rsf, bias, outputs
-    float* logits_out; // (M, 256) fp32 or nullptr
-    int num_kb;        // K / 64
-    int kb_per_split;
+    RouteArgs route;    // M, E, G, TG, K (topk), group_kind, renorm, rsf, bias, outputs
+    float* logits_out;  // (M, 256) fp32 or nullptr
+    int num_kb;         // K / 64
+    int kb_per_split;   // k-blocks per CTA
+    int ncl;            // clusters per tile whose partials meet in the workspace (1: none)
+    float* ws_part;     // [ncl][M][256] fp32 cluster partials (ncl > 1)
+    unsigned int* ws_ticket;  // [SPLIT] arrival counters, zero between calls (ncl > 1)
 };
+
+// Workspace of the wide split-K path (one 128-row tile over several clusters).
+constexpr int kWideSplit = 8;     // CTAs per cluster on that path
+constexpr int kWideMaxClusters = 18;
+constexpr int kWideMinKb = 16;    // k-blocks below which one cluster suffices
+
+__host__ __device__ constexpr int wide_clusters(int num_kb) {
+    const int c = (num_kb + kWideSplit - 1) / kWideSplit;
+    return c > kWideMaxClusters ? kWideMaxClusters : c;
+}
+
+size_t wide_workspace_bytes(int64_t M, int num_kb) {
+    const size_t part = (size_t)wide_clusters(num_kb) * (size_t)M * kBN * sizeof(float);
+    return (part + 255) / 256 * 256 + 256;
+}
 
 __host__ __device__ constexpr size_t fused_smem_bytes() {
     return 1024 + (size_t)kStages * kStageBytes + Router::BIAS_FLOATS * 4 + 256;
@@ -77,7 +95,7 @@ struct FinScores {
     }
 };
 
-template <int SPLIT, bool B_MN_MAJOR, bool BIAS>
+template <int SPLIT, bool B_MN_MAJOR, bool BIAS, bool GRED>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_router_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         FusedArgs fa) {
@@ -93,22 +111,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* s_peer_abort = s_abort + 1;
+    volatile int* s_last = s_abort + 2;  // this CTA reduces the clusters' partials
     // Overlays of the stage ring, valid once the main loop is over: one slot
     // of partial sums per source CTA for the rows this CTA owns, in the
     // chunked staged-row layout; slot 0 is summed in place and then holds
     // the logits that are routed.
     float* slots = reinterpret_cast<float*>(smem);                                // [SPLIT][ROWS][292]
     float* fin = slots;
-    // Router scratch reuses slots 1.. once they have been summed into slot 0.
+    // Router scratch reuses slots 1.. (and the rest of the ring) once they
+    // have been summed into slot 0.
     auto* scratch = reinterpret_cast<typename R_t::Scratch*>(slots + (size_t)ROWS * kFinStride);
-    static_assert((size_t)(SPLIT - 1) * ROWS * kFinStride * 4 >= kEpiWarps * sizeof(typename R_t::Scratch),
-                  "router scratch must fit in the summed slots");
+    static_assert((size_t)ROWS * kFinStride * 4 + kEpiWarps * sizeof(typename R_t::Scratch) <=
+                      (size_t)kStages * kStageBytes,
+                  "router scratch must fit in the stage ring");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = ptx::cluster_ctarank();
-    const int m_tile = blockIdx.x / SPLIT;
-    const int kb0 = (int)rank * fa.kb_per_split;
+    const int cl = GRED ? (int)((blockIdx.x / SPLIT) % fa.ncl) : 0;   // cluster within the tile
+    const int m_tile = GRED ? (int)(blockIdx.x / (SPLIT * fa.ncl)) : (int)(blockIdx.x / SPLIT);
+    const int kb0 = (cl * SPLIT + (int)rank) * fa.kb_per_split;
     int nkb = fa.num_kb - kb0;
     if (nkb > fa.kb_per_split) nkb = fa.kb_per_split;
     if (nkb < 0) nkb = 0;
@@ -122,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(accum, 1);
         *s_abort = 0;
         *s_peer_abort = 0;
+        *s_last = 1;
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
@@ -215,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the stage ring can be reused as the receive buffer.
     ptx::cluster_sync();
 
-    const int q = warp & 3;                 // TMEM lane quarter of this warp (warps 2..9 -> 2,3,0,1,2,3,0,1)
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int r = q * 32 + lane;            // tile row of this thread's TMEM lane
     const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const bool epi = warp >= 2;
@@ -227,9 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int owner = r / ROWS;
         const uint32_t dst = ptx::map_to_rank(
             ptx::smem_u32(slots + ((size_t)rank * ROWS + (r - owner * ROWS)) * kFinStride), owner);
-        const int half = (warp - 2) >> 2;  // which half of the columns this warp moves
+        constexpr int PARTS = kEpiWarps / 4;           // warps per TMEM lane quarter
+        constexpr int CPP = (kBN / 32) / PARTS;        // 32-column chunks per warp
+        const int part = (warp - 2) >> 2;
+        const bool live = (int64_t)m_tile * kBM + r < fa.route.M;  // rows past M carry nothing
 #pragma unroll 1
-        for (int c = half * (kBN / 64); c < (half + 1) * (kBN / 64); ++c) {
+        for (int c = part * CPP; c < (part + 1) * CPP; ++c) {
             float v[32];
             __syncwarp();
             if (has_acc) {
@@ -238,11 +264,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.0f;
             }
+            if (live) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                ptx::st_cluster_f32x4(dst + (c * 36 + 4 * i) * 4, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                for (int i = 0; i < 8; ++i)
+                    ptx::st_cluster_f32x4(dst + (c * 36 + 4 * i) * 4, v[4 * i], v[4 * i + 1], v[4 * i + 2],
+                                          v[4 * i + 3]);
+            }
         }
-        if (*s_abort && half == 0)
+        if (*s_abort && part == 0)
             ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(const_cast<int*>(s_peer_abort)), owner), 1u);
     }
     ptx::cluster_sync();
@@ -259,6 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int col = col0; col < col0 + COLS; col += 4) {
             const int off = lr * kFinStride + (col >> 5) * 36 + (col & 31);
+            if (grow >= fa.route.M) {
+                *reinterpret_cast<float4*>(slots + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+                continue;
+            }
             float4 acc = *reinterpret_cast<const float4*>(slots + off);
             for (int src = 1; src < SPLIT; ++src) {
                 const float4 v = *reinterpret_cast<const float4*>(slots + (size_t)src * ROWS * kFinStride + off);
@@ -268,8 +301,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc.w += v.w;
             }
             *reinterpret_cast<float4*>(slots + off) = acc;
-            if (fa.logits_out != nullptr && grow < fa.route.M)
+            if (!GRED && fa.logits_out != nullptr && grow < fa.route.M)
                 *reinterpret_cast<float4*>(fa.logits_out + grow * kBN + col) = acc;
+        }
+    }
+    if constexpr (GRED) {
+        // Across clusters: publish this cluster's partial of the owned rows;
+        // the last cluster to arrive sums all of them in cluster order.
+        if (epi) {
+            constexpr int COLS = kBN * ROWS / (kEpiWarps * 32);
+            const int t = threadIdx.x - 64;
+            const int lr = t % ROWS;
+            const int col0 = (t / ROWS) * COLS;
+            const int64_t grow = row_base + lr;
+            if (grow < fa.route.M) {
+                float* dst = fa.ws_part + ((size_t)cl * fa.route.M + grow) * kBN;
+                for (int col = col0; col < col0 + COLS; col += 4)
+                    *reinterpret_cast<float4*>(dst + col) =
+                        *reinterpret_cast<const float4*>(slots + lr * kFinStride + (col >> 5) * 36 + (col & 31));
+            }
+            ptx::named_barrier_sync(1, kEpiWarps * 32);
+            if (t == 0) {
+                __threadfence();  // the block's partial writes, ordered by the barrier, before the ticket
+                *s_last = (atomicAdd(&fa.ws_ticket[rank], 1u) == (unsigned)(fa.ncl - 1)) ? 1 : 0;
+            }
+            ptx::named_barrier_sync(1, kEpiWarps * 32);
+            if (*s_last) {
+                __threadfence();
+                for (int col = col0; col < col0 + COLS; col += 4) {
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (grow < fa.route.M) {
+                        // gather 6 partials at a time, add them in cluster order
+                        for (int g0 = 0; g0 < fa.ncl; g0 += 6) {
+                            float4 part[6];
+#pragma unroll
+                            for (int j = 0; j < 6; ++j)
+                                if (g0 + j < fa.ncl)
+                                    part[j] = __ldcg(reinterpret_cast<const float4*>(
+                                        fa.ws_part + ((size_t)(g0 + j) * fa.route.M + grow) * kBN + col));
+#pragma unroll
+                            for (int j = 0; j < 6; ++j) {
+                                if (g0 + j < fa.ncl) {
+                                    acc.x += part[j].x;
+                                    acc.y += part[j].y;
+                                    acc.z += part[j].z;
+                                    acc.w += part[j].w;
+                                }
+                            }
+                        }
+                        if (fa.logits_out != nullptr)
+                            *reinterpret_cast<float4*>(fa.logits_out + grow * kBN + col) = acc;
+                    }
+                    *reinterpret_cast<float4*>(slots + lr * kFinStride + (col >> 5) * 36 + (col & 31)) = acc;
+                }
+                if (t == 0) fa.ws_ticket[rank] = 0u;  // ready for the next call
+            }
         }
     }
     ptx::tc_fence_before();
@@ -279,8 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_dealloc(tmem, 256);
     }
 
-    // Routing of the owned rows by the four epilogue warps (4 rows each).
-    if (epi) {
+    // Routing of the owned rows by the epilogue warps (4 rows each per pass).
+    if (epi && *s_last) {
         const bool aborted = *s_abort || *s_peer_abort;
         const int ew = warp - 2;
         const int seg = lane / R_t::L;
@@ -313,10 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int SPLIT, bool B_MN, bool BIAS>
+template <int SPLIT, bool B_MN, bool BIAS, bool GRED = false>
 int launch_fused(const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs& fa, int m_tiles,
                  cudaStream_t stream) {
-    auto kern = fused_router_kernel<SPLIT, B_MN, BIAS>;
+    auto kern = fused_router_kernel<SPLIT, B_MN, BIAS, GRED>;
     {
         static std::mutex mu;
         static bool done[64] = {};
@@ -335,7 +421,7 @@ int launch_fused(const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs
         }
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(m_tiles * SPLIT), 1, 1);
+    cfg.gridDim = dim3((unsigned)(m_tiles * SPLIT * fa.ncl), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = fused_smem_bytes();
     cfg.stream = stream;
@@ -371,7 +457,7 @@ int max_schedulable_split(int dev) {
     std::lock_guard<std::mutex> lk(mu);
     if (cached[dev & 63]) return cached[dev & 63];
     int best = 8;
-    auto kern = fused_router_kernel<16, false, true>;
+    auto kern = fused_router_kernel<16, false, true, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem_bytes()) ==
             cudaSuccess &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
@@ -410,6 +496,10 @@ extern "C" {
 
 size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E) {
     if (M < 0 || K < 1 || E < 1) return (size_t)-1;
+    // A single 128-token tile with a long K spreads K over several clusters
+    // whose partial sums meet in the workspace; larger batches need none.
+    if (M >= 1 && M <= moe::kBM && E == 256 && K % 64 == 0 && K / 64 >= moe::kWideMinKb)
+        return moe::wide_workspace_bytes(M, K / 64);
     return 0;
 }
 
@@ -419,8 +509,6 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
                           int32_t topk_group, float routed_scaling_factor, float* topk_weights,
                           int32_t* topk_ids, float* logits_out, void* workspace,
                           size_t workspace_bytes, void* stream) {
-    (void)workspace;
-    (void)workspace_bytes;
     using namespace moe;
     const char* who = "moe_fused_router_topk";
     char msg[256];
@@ -485,6 +573,13 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
 
     const int m_tiles = (int)((M + kBM - 1) / kBM);
     const int num_kb = K / kBK;
+    const size_t ws_need = moe_fused_router_workspace_size(M, K, E);
+    if (ws_need > 0 && (workspace == nullptr || workspace_bytes < ws_need ||
+                        (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)) {
+        snprintf(msg, sizeof msg, "%s: needs a 256-byte aligned workspace of %zu bytes (got %zu)", who, ws_need,
+                 workspace_bytes);
+        return set_error(MOE_ERR_INVALID_ARG, msg);
+    }
     int split = 2;
     const int per = sms / (m_tiles > 0 ? m_tiles : 1);
     if (per >= 16) split = 16;
@@ -509,7 +604,25 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
     fa.logits_out = logits_out;
     fa.num_kb = num_kb;
     fa.kb_per_split = (num_kb + split - 1) / split;
+    fa.ncl = 1;
+    fa.ws_part = nullptr;
+    fa.ws_ticket = nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (ws_need > 0) {
+        // wide split-K: ncl clusters of kWideSplit CTAs, one CTA per SM
+        int ncl = wide_clusters(num_kb);
+        if (ncl > sms / kWideSplit) ncl = sms / kWideSplit;
+        if (ncl < 1) ncl = 1;
+        fa.ncl = ncl;
+        fa.kb_per_split = (num_kb + ncl * kWideSplit - 1) / (ncl * kWideSplit);
+        fa.ws_part = static_cast<float*>(workspace);
+        fa.ws_ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + ws_need - 256);
+        if (b_mn)
+            return correction_bias ? launch_fused<kWideSplit, true, true, true>(tmA, tmB, fa, m_tiles, st)
+                                   : launch_fused<kWideSplit, true, false, true>(tmA, tmB, fa, m_tiles, st);
+        return correction_bias ? launch_fused<kWideSplit, false, true, true>(tmA, tmB, fa, m_tiles, st)
+                               : launch_fused<kWideSplit, false, false, true>(tmA, tmB, fa, m_tiles, st);
+    }
     if (b_mn)
         return correction_bias ? launch_split<true, true>(split, tmA, tmB, fa, m_tiles, st)
                                : launch_split<true, false>(split, tmA, tmB, fa, m_tiles, st);

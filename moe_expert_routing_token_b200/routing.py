@@ -206,7 +206,8 @@ def fused_router_topk(hidden_states: torch.Tensor, router_weight: torch.Tensor, 
     logits = torch.empty(M, E, dtype=torch.float32, device=dev) if return_logits else None
     need = fused_router_workspace_size(M, K, E)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        # the workspace must start zeroed; the library leaves it zeroed again
+        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
     wsp = workspace.data_ptr() if (need and workspace is not None) else None
     st = lib().moe_fused_router_topk(hidden_states.data_ptr(), router_weight.data_ptr(), layout, bp, M,
                                      K, E, topk, int(bool(renormalize)), num_expert_group, topk_group,

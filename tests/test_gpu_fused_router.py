@@ -125,6 +125,39 @@ def test_deterministic_across_calls():
     assert all(torch.equal(x, y) for x, y in zip(a, c))
 
 
+@pytest.mark.parametrize("M", [1, 7, 64, 128])
+def test_wide_split_path_reuses_its_workspace(M):
+    """Single-tile batches spread K over several clusters that meet in the
+    workspace; the arrival counters must be back at zero after every call,
+    so back-to-back calls on one workspace give identical results."""
+    K = 7168
+    need = moe.fused_router_workspace_size(M, K, 256)
+    assert need > 0
+    h, w, b = _draw(M, K, seed=11 + M)
+    hd, wd, bd = h.to(DEV), w.to(DEV), b.to(DEV)
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    outs = [moe.fused_router_topk(hd, wd, bd, 8, True, 8, 4, 2.5, return_logits=True, workspace=ws)
+            for _ in range(3)]
+    torch.cuda.synchronize()
+    tail = ws[need - 256:]
+    assert int(tail.sum()) == 0, "arrival counters not reset"
+    for o in outs[1:]:
+        assert all(torch.equal(x, y) for x, y in zip(outs[0], o))
+    _check(h, w, b, "ke")
+
+
+def test_wide_split_needs_workspace():
+    h = torch.zeros(64, 7168, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(7168, 256, dtype=torch.bfloat16, device=DEV)
+    weights = torch.empty(64, 8, device=DEV)
+    ids = torch.empty(64, 8, dtype=torch.int32, device=DEV)
+    L = moe.lib()
+    st = L.moe_fused_router_topk(h.data_ptr(), w.data_ptr(), 0, None, 64, 7168, 256, 8, 1, 8, 4, 2.5,
+                                 weights.data_ptr(), ids.data_ptr(), None, None, 0,
+                                 torch.cuda.current_stream().cuda_stream)
+    assert st == 1 and b"workspace" in L.moe_last_error()
+
+
 def test_invalid_arguments():
     h = torch.zeros(4, 100, dtype=torch.bfloat16, device=DEV)
     w = torch.zeros(100, 256, dtype=torch.bfloat16, device=DEV)
