@@ -197,6 +197,44 @@ MOE_API int moe_fused_router_topk(const void* hidden_states, const void* router_
                           float* logits_out, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/*
+ * moe_fused_router_topk_noalloc - moe_fused_router_topk for callers that
+ * cannot hand the library a workspace.  (The routing pages have no
+ * counterpart to this call; it exists for the library's users.)
+ *
+ * Who needs it: code that is not allowed to allocate device memory at the
+ * point where it routes tokens - inference engines that reserve every byte
+ * of device memory during start-up and forbid allocations afterwards, or
+ * plugin and embedding hosts that give the extension no allocator at all.
+ * Batches of up to 128 tokens with a long hidden size need scratch memory
+ * (moe_fused_router_workspace_size() > 0); this entry point takes it from a
+ * fixed 2 MiB array compiled into the library instead of from the caller.
+ *
+ *   Arguments, layouts and results are those of moe_fused_router_topk,
+ *   without `workspace` / `workspace_bytes`.
+ *   Limit: sizes whose workspace would exceed 2 MiB are rejected with
+ *   MOE_ERR_UNSUPPORTED and a message naming the sizes.  With K = 7168 every
+ *   M fits (at most 1.75 MiB); K >= 9216 with M close to 128 does not.
+ *   Batches above 128 tokens need no scratch and always work.
+ *   Memory: nothing is allocated or freed.  Every GPU that loads the library
+ *   keeps the 2 MiB array for the life of the process.  The first call on
+ *   each device looks up the array's device address (cudaGetSymbolAddress);
+ *   make that first call before capturing the stream into a CUDA graph.
+ *   Each call clears the array's 256 bytes of arrival counters on `stream`
+ *   (cudaMemsetAsync) before launching.
+ *   Concurrency: all calls on a device share the one array, which keeps the
+ *   last call's partial sums; calls that overlap on the GPU (different
+ *   streams, or host threads racing on one device) race on it and give wrong
+ *   results.  Serialise them (one stream), or use moe_fused_router_topk with a
+ *   workspace per stream.
+ */
+MOE_API int moe_fused_router_topk_noalloc(const void* hidden_states, const void* router_weight,
+                                          int weight_layout, const float* correction_bias, int64_t M,
+                                          int32_t K, int32_t E, int32_t topk, int32_t renormalize,
+                                          int32_t num_expert_group, int32_t topk_group,
+                                          float routed_scaling_factor, float* topk_weights,
+                                          int32_t* topk_ids, float* logits_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -482,6 +482,33 @@ int max_schedulable_split(int dev) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch for moe_fused_router_topk_noalloc: a fixed device array that every
+// GPU loading this library holds until the process exits.  Host code must not
+// use the symbol itself as a pointer (on the host it only names the
+// variable); its device address is looked up per device.
+constexpr size_t kNoAllocScratchBytes = 2u << 20;  // 2 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up on
+// the first call per device.
+int noalloc_scratch(void** ptr) {
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return set_cuda_error(err, "cudaGetDevice");
+    std::lock_guard<std::mutex> lk(mu);
+    if (addr[dev & 63] == nullptr) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (err != cudaSuccess) return set_cuda_error(err, "cudaGetSymbolAddress(no-alloc scratch)");
+        addr[dev & 63] = p;
+    }
+    *ptr = addr[dev & 63];
+    return MOE_OK;
+}
+
 int read_fused_watchdog(unsigned int* count) {
     unsigned int v = 0;
     cudaError_t err = cudaMemcpyFromSymbol(&v, g_watchdog_trips_fused, sizeof(v));
@@ -628,6 +655,39 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
                                : launch_split<true, false>(split, tmA, tmB, fa, m_tiles, st);
     return correction_bias ? launch_split<false, true>(split, tmA, tmB, fa, m_tiles, st)
                            : launch_split<false, false>(split, tmA, tmB, fa, m_tiles, st);
+}
+
+int moe_fused_router_topk_noalloc(const void* hidden_states, const void* router_weight, int weight_layout,
+                                  const float* correction_bias, int64_t M, int32_t K, int32_t E,
+                                  int32_t topk, int32_t renormalize, int32_t num_expert_group,
+                                  int32_t topk_group, float routed_scaling_factor, float* topk_weights,
+                                  int32_t* topk_ids, float* logits_out, void* stream) {
+    using namespace moe;
+    const size_t need = moe_fused_router_workspace_size(M, K, E);
+    if (need == (size_t)-1)
+        return set_error(MOE_ERR_INVALID_ARG, "moe_fused_router_topk_noalloc: invalid sizes");
+    if (need > kNoAllocScratchBytes) {
+        char msg[256];
+        snprintf(msg, sizeof msg,
+                 "moe_fused_router_topk_noalloc: M=%lld, K=%d need %zu bytes of scratch; the built-in "
+                 "scratch holds %zu (use moe_fused_router_topk with a workspace)",
+                 (long long)M, K, need, kNoAllocScratchBytes);
+        return set_error(MOE_ERR_UNSUPPORTED, msg);
+    }
+    void* scratch = nullptr;
+    if (need > 0) {
+        int rc = noalloc_scratch(&scratch);
+        if (rc != MOE_OK) return rc;
+        // The arrival counters at the end of the scratch must start at zero;
+        // clear them on the call's stream (a previous call that stopped early
+        // could have left them set).
+        cudaError_t err = cudaMemsetAsync(static_cast<char*>(scratch) + need - 256, 0, 256,
+                                          static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return set_cuda_error(err, "cudaMemsetAsync(no-alloc scratch counters)");
+    }
+    return moe_fused_router_topk(hidden_states, router_weight, weight_layout, correction_bias, M, K, E, topk,
+                                 renormalize, num_expert_group, topk_group, routed_scaling_factor, topk_weights,
+                                 topk_ids, logits_out, scratch, need, stream);
 }
 
 }  // extern "C"

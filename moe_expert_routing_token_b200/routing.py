@@ -44,6 +44,8 @@ SIGNATURES = {
     "moe_fused_router_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_fused_router_topk": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32, _i32,
                                              _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_fused_router_topk_noalloc": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32,
+                                                     _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
 }
 
 
