@@ -18,6 +18,7 @@
 #include "moe_routing.h"
 #include "routing_kernels.cuh"
 #include "routing_staged.cuh"
+#include "routing_stream.cuh"
 #include "tma_host.cuh"
 
 namespace moe {
@@ -129,42 +130,70 @@ int launch_segment(int E, const RouteArgs& a, cudaStream_t st) {
 // Batches at least this large take the TMA-staged streaming kernel.
 constexpr int64_t kStagedMinRows = 1024;
 
-template <typename TIn, int E, int C, int SCORE, bool BIAS>
-int launch_staged_ec(const RouteArgs& a, cudaStream_t st) {
-    using Cfg = StagedCfg<TIn, E, C, SCORE, BIAS>;
-    auto kern = route_staged_kernel<TIn, E, C, SCORE, BIAS>;
-    const int threads = (Cfg::W + 1) * 32;
+// Launch a persistent TMA-ring routing kernel: raise its dynamic shared
+// memory limit once per (kernel, device), encode the logits tensor map
+// (boxes of box_e x rb elements, 128-byte swizzle) and size the grid to the
+// resident blocks.
+using RingKernel = void (*)(const CUtensorMap, RouteArgs, int64_t);
+
+template <typename TIn>
+int launch_ring(RingKernel kern, size_t smem, int threads, int box_e, int rb, const RouteArgs& a,
+                cudaStream_t st, const char* what) {
     int dev = 0, sms = 0, per_sm = 1;
     int rc = device_and_sms(&dev, &sms);
     if (rc != MOE_OK) return rc;
     {
-        // raise the dynamic shared memory limit once per device
         static std::mutex mu;
-        static bool done[64] = {};
+        static std::unordered_map<const void*, uint64_t> done;  // kernel -> devices done (bit mask)
         std::lock_guard<std::mutex> lk(mu);
-        if (!done[dev & 63]) {
-            cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)Cfg::SMEM);
-            if (err != cudaSuccess) return cuda_fail(err, "cudaFuncSetAttribute(staged routing)");
-            done[dev & 63] = true;
+        uint64_t& bits = done[reinterpret_cast<const void*>(kern)];
+        if (!(bits & (1ull << (dev & 63)))) {
+            cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (err != cudaSuccess) return cuda_fail(err, what);
+            bits |= 1ull << (dev & 63);
         }
     }
-    rc = resident_blocks(dev, kern, threads, Cfg::SMEM, &per_sm);
+    rc = resident_blocks(dev, kern, threads, smem, &per_sm);
     if (rc != MOE_OK) return rc;
     CUtensorMap tmap;
     cudaError_t err = encode_tmap_2d(&tmap, a.logits,
                                      sizeof(TIn) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                                     (uint64_t)a.M, (uint64_t)E, (uint64_t)E * sizeof(TIn), Cfg::BOX_E,
-                                     Cfg::RB, true);
+                                     (uint64_t)a.M, (uint64_t)a.E, (uint64_t)a.E * sizeof(TIn), box_e, rb, true);
     if (err != cudaSuccess) return cuda_fail(err, "cuTensorMapEncodeTiled(logits)");
-    const int64_t nblocks = (a.M + Cfg::RB - 1) / Cfg::RB;
+    const int64_t nblocks = (a.M + rb - 1) / rb;
     const int64_t cap = (int64_t)sms * per_sm;
     const int grid = (int)(nblocks < cap ? nblocks : cap);
-    kern<<<grid, threads, Cfg::SMEM, st>>>(tmap, a, nblocks);
+    kern<<<grid, threads, smem, st>>>(tmap, a, nblocks);
     err = cudaGetLastError();
-    if (err != cudaSuccess) return cuda_fail(err, "staged routing kernel launch");
+    if (err != cudaSuccess) return cuda_fail(err, what);
     return MOE_OK;
+}
+
+template <typename TIn, int E, int C, int SCORE, bool BIAS>
+int launch_staged_ec(const RouteArgs& a, cudaStream_t st) {
+    using Cfg = StagedCfg<TIn, E, C, SCORE, BIAS>;
+    return launch_ring<TIn>(route_staged_kernel<TIn, E, C, SCORE, BIAS>, Cfg::SMEM, (Cfg::W + 1) * 32,
+                            Cfg::BOX_E, Cfg::RB, a, st, "staged routing kernel");
+}
+
+template <typename TIn, int E, int C, int SCORE, bool BIAS, bool APPROX>
+int launch_stream_ec(const RouteArgs& a, cudaStream_t st) {
+    using Cfg = StreamCfg<TIn, E, C, SCORE, BIAS, APPROX>;
+    return launch_ring<TIn>(route_stream_kernel<TIn, E, C, SCORE, BIAS, APPROX>, Cfg::SMEM,
+                            kStreamThreads, Cfg::BOX_E, Cfg::RB, a, st, "streaming routing kernel");
+}
+
+// Two-phase streaming kernel (topk <= 8).  The approximate phase-1 key is
+// used for sigmoid scoring when every group is kept.
+template <typename TIn, int SCORE, bool BIAS>
+int launch_stream(int E, const RouteArgs& a, cudaStream_t st) {
+    const bool approx = (SCORE == kSigmoid) && a.TG == a.G;
+    if (E == 256)
+        return approx ? launch_stream_ec<TIn, 256, 32, SCORE, BIAS, SCORE == kSigmoid>(a, st)
+                      : launch_stream_ec<TIn, 256, 32, SCORE, BIAS, false>(a, st);
+    return approx ? launch_stream_ec<TIn, 160, 20, SCORE, BIAS, SCORE == kSigmoid>(a, st)
+                  : launch_stream_ec<TIn, 160, 20, SCORE, BIAS, false>(a, st);
 }
 
 template <typename TIn, int SCORE, bool BIAS>
@@ -201,7 +230,8 @@ int dispatch_typed(const RouteArgs& a, cudaStream_t st) {
         const size_t chunk = C * esz;
         const size_t vec = (chunk % 16 == 0) ? 16 : 8;
         if (a.M >= kStagedMinRows && aligned(a.logits, 16) && (E * esz) % 16 == 0)
-            return launch_staged<TIn, SCORE, BIAS>(E, a, st);
+            return (a.K <= 8 && (E == 160 || kC256 == 32)) ? launch_stream<TIn, SCORE, BIAS>(E, a, st)
+                                                          : launch_staged<TIn, SCORE, BIAS>(E, a, st);
         if (aligned(a.logits, vec)) return launch_segment<TIn, SCORE, BIAS>(E, a, st);
     }
     if ((E == 8 || E == 16 || E == 32) && aligned(a.logits, 16))

@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int ROWS = kBM / SPLIT;  // rows of the tile this CTA routes
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = ptx::smem_align<1024>(smem_raw);
     float* s_bias = reinterpret_cast<float*>(smem + (size_t)kStages * kStageBytes);
     uint64_t* full = reinterpret_cast<uint64_t*>(s_bias + Router::BIAS_FLOATS);
     uint64_t* empty = full + kStages;

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32)
     constexpr int W = Cfg::W, R = Cfg::R, RB = Cfg::RB, S = Cfg::S, L = Router::L;
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = ptx::smem_align<1024>(smem_raw);
     uint8_t* stages = base;
     auto* scratch = reinterpret_cast<typename Router::Scratch*>(stages + (size_t)S * Cfg::STAGE_BYTES);
     float* s_bias = reinterpret_cast<float*>(scratch + W);

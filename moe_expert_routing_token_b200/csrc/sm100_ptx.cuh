@@ -216,6 +216,16 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+// Round a dynamic shared-memory pointer up to ALIGN bytes by adding an offset
+// to it.  (Going through an integer cast instead loses the pointer's address
+// space: every access through it then compiles to a generic load or store,
+// with global-memory latency.)
+template <int ALIGN>
+__device__ __forceinline__ uint8_t* smem_align(uint8_t* p) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    return p + ((ALIGN - (a & (ALIGN - 1))) & (ALIGN - 1));
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

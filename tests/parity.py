@@ -9,9 +9,15 @@ all margins are measured by the oracle in double precision):
   the *selected* experts are themselves within ``eps`` of each other, the
   order inside that run is free but the id set must still match exactly.
 * Other rows are *near-tie* rows: counted, and accepted when the ids are
-  unique, every id lies in a group scoring >= gs_(TG) - eps, every chosen
-  expert scores >= s_(k) - eps, and every oracle pick the GPU left out
-  scores <= s_(k) + eps.
+  unique, every id lies in a group scoring >= gs_(TG) - eps, and the choice
+  is a top-k within eps inside the groups kept:
+  - group margin clear (the GPU keeps the oracle's groups): every chosen
+    expert scores >= s_(k) - eps and every oracle pick the GPU left out
+    scores <= s_(k) + eps;
+  - group margin within eps (another set of groups is as valid): the GPU's
+    groups plus the clearly kept ones (gs > gs_(TG) + eps) number at most
+    TG, and no expert of those groups that the GPU left out scores more than
+    eps above the GPU's weakest pick.
 * Weights are compared per slot against the oracle's unbiased score of the
   expert the GPU chose, renormalised over the GPU's chosen set and scaled:
   |dw| <= 1e-6 for fp32 logits, |dw| <= 2e-3 |w| for bf16 logits (a 1e-30
@@ -101,12 +107,21 @@ def compare(w_gpu, ids_gpu, orc, *, E: int, G: int, TG: int, k: int, renorm: boo
         gs_tg = np.sort(gs[r])[::-1][TG - 1]
         if np.any(gs[r, ids // S] < gs_tg - eps):
             rep.failures.append(f"row {r} (near tie): id in a dropped group {ids.tolist()}")
-        s_k = s[r, ids_o[r, k - 1]]
-        if np.any(s[r, ids] < s_k - eps):
-            rep.failures.append(f"row {r} (near tie): chose an expert below s_(k) - eps")
-        omitted = np.setdiff1d(ids_o[r], ids)
-        if omitted.size and np.any(s[r, omitted] > s_k + eps):
-            rep.failures.append(f"row {r} (near tie): left out an expert above s_(k) + eps")
+        if d_grp[r] > eps:
+            s_k = s[r, ids_o[r, k - 1]]
+            if np.any(s[r, ids] < s_k - eps):
+                rep.failures.append(f"row {r} (near tie): chose an expert below s_(k) - eps")
+            omitted = np.setdiff1d(ids_o[r], ids)
+            if omitted.size and np.any(s[r, omitted] > s_k + eps):
+                rep.failures.append(f"row {r} (near tie): left out an expert above s_(k) + eps")
+        else:
+            kept = set((ids // S).tolist()) | set(np.nonzero(gs[r] > gs_tg + eps)[0].tolist())
+            if len(kept) > TG:
+                rep.failures.append(f"row {r} (group near tie): {len(kept)} groups kept > {TG}")
+            members = np.concatenate([np.arange(g * S, (g + 1) * S) for g in sorted(kept)])
+            others = np.setdiff1d(members, ids)
+            if others.size and np.any(s[r, others] > s[r, ids].min() + eps):
+                rep.failures.append(f"row {r} (group near tie): left out a better expert of a kept group")
 
     # weights for the GPU's choice
     pw = np.take_along_axis(p, ids_gpu, axis=1)
