@@ -104,10 +104,13 @@ def measured_peaks() -> dict:
             "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files=None) -> str:
+    """sha256 prefix of the kernel sources (all csrc/*.cu{,h}, or the listed
+    files, in sorted order)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "moe_expert_routing_token_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    names = sorted(files) if files else sorted(os.listdir(csrc))
+    for f in names:
         if f.endswith((".cu", ".cuh")):
             h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
@@ -115,14 +118,17 @@ def kernel_source_hash() -> str:
 
 def profiled_traffic(name: str, M: int):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the current kernel sources (else None).  The summary names the source files
+    its kernel is built from (``kernel_sources:``) and their hash."""
     path = os.path.join(ROOT, "profiles", f"traffic_{name}_M{M}.txt")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     src = re.search(r"kernel_source_sha:\s*(\w+)", text)
     val = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not src or not val or src.group(1) != kernel_source_hash():
+    files = re.search(r"kernel_sources:\s*(.+)", text)
+    files = files.group(1).split() if files else None
+    if not src or not val or src.group(1) != kernel_source_hash(files):
         return None
     return float(val.group(1))
 
@@ -213,6 +219,30 @@ def time_oracle(name: str, M: int, seconds: float) -> dict:
                       f"M={M} draw), single-threaded C oracle in double, {el:.1f} s"}
 
 
+# ---------------------------------------------------------------------------
+# Multi-rank host logic (no data-path collective: each rank routes its own rows)
+def rank_seed(name: str, M: int, rank: int) -> int:
+    """Each rank draws its own batch of the workload (rows sharded by rank)."""
+    from moe_expert_routing_token_b200 import inputs
+    return inputs.default_seed(name, M) + 7919 * rank
+
+
+def job_elapsed_ms(local_ms: float, world: int, device) -> float:
+    """The job's time: the maximum of the ranks' device-timed elapsed times."""
+    if world == 1:
+        return float(local_ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(M: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the tokens every rank routed over the job time."""
+    return M * steps * world / (ms / 1e3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -284,7 +314,7 @@ def run_ours(args):
     name = args.workload
     M = args.M or DEFAULT_M[name]
     sp = inputs.SPECS[name]
-    d = inputs.make(name, M, seed=inputs.default_seed(name, M) + 7919 * rank)
+    d = inputs.make(name, M, seed=rank_seed(name, M, rank))
     # a dedicated stream: graphs cannot be captured on the legacy default stream
     stream = torch.cuda.Stream(dev)
     torch.cuda.set_stream(stream)
@@ -375,13 +405,8 @@ def run_ours(args):
         dist.barrier()
     ms = start.elapsed_time(stop)
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-
-    tokens = M * args.steps * world
-    value = tokens / (ms / 1e3)
+    ms = job_elapsed_ms(ms, world, dev)
+    value = job_tokens_per_s(M, args.steps, world, ms)
     us_per_call = ms * 1e3 / args.steps
 
     # ---- end to end through the public API with host buffers ----------------
@@ -473,12 +498,8 @@ def e2e_measure(name, M, sp, d, dev, stream, world, args):
             step()
         b.record(stream)
         torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": M * steps * world / (ms / 1e3), "unit": "tokens/s",
+    ms = job_elapsed_ms(a.elapsed_time(b), world, dev)
+    return {"value": job_tokens_per_s(M, steps, world, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": src.numel() * src.element_size(),
             "d2h_bytes_per_step": hw.numel() * 4 + hi.numel() * 4, "steps": steps}
 
