@@ -77,8 +77,21 @@ size_t wide_workspace_bytes(int64_t M, int num_kb) {
     return (part + 255) / 256 * 256 + 256;
 }
 
+// Bytes at the start of shared memory used first as the stage ring, then (after
+// the main loop) as the split-K exchange and routing area.  With SPLIT = 2 that
+// area holds this CTA's own rows (padded staged layout), the partner's partials
+// (compact, received by one bulk copy) and the rows this CTA sends.
+// Rows of the send/receive buffers are padded to an odd number of 16-byte
+// chunks, so the 32 lanes of a warp (32 different rows) hit distinct banks.
+constexpr int kPairStride = kBN + 4;
+constexpr size_t kPairExchangeBytes =
+    (size_t)(kBM / 2) * kFinStride * 4 + 2 * (size_t)(kBM / 2) * kPairStride * 4;
+constexpr size_t kOverlayBytes = (size_t)kStages * kStageBytes > kPairExchangeBytes
+                                     ? (size_t)kStages * kStageBytes
+                                     : kPairExchangeBytes;
+
 __host__ __device__ constexpr size_t fused_smem_bytes() {
-    return 1024 + (size_t)kStages * kStageBytes + Router::BIAS_FLOATS * 4 + 256;
+    return 1024 + kOverlayBytes + Router::BIAS_FLOATS * 4 + 256;
 }
 
 // Owner-side staged logits row: chunk c (32 floats) at c * 36.
@@ -104,11 +117,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = ptx::smem_align<1024>(smem_raw);
-    float* s_bias = reinterpret_cast<float*>(smem + (size_t)kStages * kStageBytes);
+    float* s_bias = reinterpret_cast<float*>(smem + kOverlayBytes);
     uint64_t* full = reinterpret_cast<uint64_t*>(s_bias + Router::BIAS_FLOATS);
     uint64_t* empty = full + kStages;
     uint64_t* accum = empty + kStages;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
+    uint64_t* recv_bar = accum + 1;  // SPLIT = 2: the partner's partials have landed
+    uint64_t* sent_bar = accum + 2;  // SPLIT = 2: the partner holds our partials
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 3);
     volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* s_peer_abort = s_abort + 1;
     volatile int* s_last = s_abort + 2;  // this CTA reduces the clusters' partials
@@ -121,9 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Router scratch reuses slots 1.. (and the rest of the ring) once they
     // have been summed into slot 0.
     auto* scratch = reinterpret_cast<typename R_t::Scratch*>(slots + (size_t)ROWS * kFinStride);
-    static_assert((size_t)ROWS * kFinStride * 4 + kEpiWarps * sizeof(typename R_t::Scratch) <=
-                      (size_t)kStages * kStageBytes,
+    static_assert((size_t)ROWS * kFinStride * 4 + kEpiWarps * sizeof(typename R_t::Scratch) <= kOverlayBytes,
                   "router scratch must fit in the stage ring");
+    static_assert(SPLIT != 2 || kPairExchangeBytes <= kOverlayBytes, "pair exchange area");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -142,6 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&empty[s], 1);
         }
         ptx::mbar_init(accum, 1);
+        ptx::mbar_init(recv_bar, 1);
+        ptx::mbar_init(sent_bar, 1);
         *s_abort = 0;
         *s_peer_abort = 0;
         *s_last = 1;
@@ -153,13 +170,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_alloc(tmem_holder, 256);
         ptx::tmem_relinquish();
     }
-    // The prologue above overlaps the previous kernel; inputs are read after it.
-    ptx::griddep_wait();
-    if constexpr (BIAS) Router::load_bias_padded(fa.route.bias, s_bias);
     ptx::tc_fence_before();
-    __syncthreads();
+    __syncthreads();  // barriers initialised, TMEM address published
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // Everything above overlaps the previous kernel; inputs are read after it.
+    // The producer starts streaming at once; the epilogue warps load the bias
+    // meanwhile (their own barrier: they are the only readers).
+    ptx::griddep_wait();
+    if (warp >= 2) {
+        if constexpr (BIAS) {
+            for (int e = threadIdx.x - 64; e < 256; e += kEpiWarps * 32)
+                s_bias[(e / 32) * Router::CS + e % 32] = __ldg(fa.route.bias + e);
+        }
+        ptx::named_barrier_sync(2, kEpiWarps * 32);
+    }
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
@@ -243,38 +268,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const bool epi = warp >= 2;
     const bool has_acc = nkb > 0;           // uniform over the CTA
-    if (epi) {
+    float* const recv = slots + (size_t)ROWS * kFinStride;  // SPLIT = 2: partner's partials [ROWS][260]
+    float* const send = recv + (size_t)ROWS * kPairStride;  // SPLIT = 2: rows the partner owns [ROWS][260]
+    if constexpr (SPLIT == 2 && !GRED) {
+        // Own rows go to the staged layout, the partner's rows to a compact
+        // send buffer that one bulk copy moves into the partner's receive
+        // area (16-byte stores across the cluster are far slower).
+        if (epi) {
+            const int owner = r / ROWS;
+            const int lr = r - owner * ROWS;
+            const int part = (warp - 2) >> 2;
+            const int c0 = part * 2;  // two 32-column chunks per warp
+            const bool live = (int64_t)m_tile * kBM + r < fa.route.M;
+            float v[64];
+            __syncwarp();
+            if (has_acc) {
+                ptx::tmem_ld64(t_row + c0 * 32, v);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) v[i] = 0.0f;
+            }
+            if (live) {
+                if (owner == (int)rank) {
+                    float* row = slots + (size_t)lr * kFinStride;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        *reinterpret_cast<float4*>(row + (c0 + i / 8) * 36 + 4 * (i % 8)) =
+                            make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                } else {
+                    float* row = send + (size_t)lr * kPairStride + c0 * 32;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        *reinterpret_cast<float4*>(row + 4 * i) =
+                            make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::named_barrier_sync(3, kEpiWarps * 32);
+            const uint32_t peer = rank ^ 1u;
+            if (threadIdx.x == 64) {
+                constexpr uint32_t kBytes = ROWS * kPairStride * 4;
+                ptx::mbar_arrive_expect_tx(recv_bar, kBytes);
+                const uint32_t dst = ptx::map_to_rank(ptx::smem_u32(recv), peer);
+                const uint32_t mb = ptx::map_to_rank(ptx::smem_u32(recv_bar), peer);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    ptx::bulk_copy_to_cluster(dst + i * (kBytes / 4), ptx::smem_u32(send) + i * (kBytes / 4),
+                                              kBytes / 4, mb);
+            }
+            if (!ptx::mbar_wait(recv_bar, 0, kWaitNs)) {
+                if (threadIdx.x == 64) atomicAdd(&g_watchdog_trips_fused, 1u);
+                *s_abort = 1;
+            }
+            // the partner's partials are here: its send buffer may be reused
+            if (threadIdx.x == 64) ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_u32(sent_bar), peer));
+        }
+    } else if (epi) {
         // Every tile row's partial sums go to slot `rank` of the CTA that
         // owns the row (this CTA included).  tcgen05.ld is warp-collective:
         // whole warps load, lanes only choose the destination.
         const int owner = r / ROWS;
-        const uint32_t dst = ptx::map_to_rank(
-            ptx::smem_u32(slots + ((size_t)rank * ROWS + (r - owner * ROWS)) * kFinStride), owner);
+        float* own_row = slots + ((size_t)rank * ROWS + (r - owner * ROWS)) * kFinStride;
+        const uint32_t dst = ptx::map_to_rank(ptx::smem_u32(own_row), owner);
         constexpr int PARTS = kEpiWarps / 4;           // warps per TMEM lane quarter
         constexpr int CPP = (kBN / 32) / PARTS;        // 32-column chunks per warp
+        static_assert(CPP == 2, "one 64-column TMEM load per epilogue warp");
         const int part = (warp - 2) >> 2;
         const bool live = (int64_t)m_tile * kBM + r < fa.route.M;  // rows past M carry nothing
-#pragma unroll 1
-        for (int c = part * CPP; c < (part + 1) * CPP; ++c) {
-            float v[32];
-            __syncwarp();
-            if (has_acc) {
-                ptx::tmem_ld32(t_row + c * 32, v);
+        const int c0 = part * CPP;
+        float v[64];
+        __syncwarp();
+        if (has_acc) {
+            ptx::tmem_ld64(t_row + c0 * 32, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = 0.0f;
+        }
+        if (live) {
+            if (owner == (int)rank) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    *reinterpret_cast<float4*>(own_row + (c0 + i / 8) * 36 + 4 * (i % 8)) =
+                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-            }
-            if (live) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    ptx::st_cluster_f32x4(dst + (c * 36 + 4 * i) * 4, v[4 * i], v[4 * i + 1], v[4 * i + 2],
-                                          v[4 * i + 3]);
+                for (int i = 0; i < 16; ++i)
+                    ptx::st_cluster_f32x4(dst + ((c0 + i / 8) * 36 + 4 * (i % 8)) * 4, v[4 * i], v[4 * i + 1],
+                                          v[4 * i + 2], v[4 * i + 3]);
             }
         }
         if (*s_abort && part == 0)
             ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(const_cast<int*>(s_peer_abort)), owner), 1u);
     }
-    ptx::cluster_sync();
+    if constexpr (SPLIT != 2 || GRED) ptx::cluster_sync();
 
     // Sum the SPLIT partials of the owned rows in rank order, all 128
     // epilogue threads in parallel, in place into slot 0.
@@ -293,12 +379,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             float4 acc = *reinterpret_cast<const float4*>(slots + off);
-            for (int src = 1; src < SPLIT; ++src) {
-                const float4 v = *reinterpret_cast<const float4*>(slots + (size_t)src * ROWS * kFinStride + off);
+            if constexpr (SPLIT == 2 && !GRED) {
+                // two partials: the sum is the same in either order
+                const float4 v = *reinterpret_cast<const float4*>(recv + (size_t)lr * kPairStride + col);
                 acc.x += v.x;
                 acc.y += v.y;
                 acc.z += v.z;
                 acc.w += v.w;
+            } else {
+                for (int src = 1; src < SPLIT; ++src) {
+                    const float4 v =
+                        *reinterpret_cast<const float4*>(slots + (size_t)src * ROWS * kFinStride + off);
+                    acc.x += v.x;
+                    acc.y += v.y;
+                    acc.z += v.z;
+                    acc.w += v.w;
+                }
             }
             *reinterpret_cast<float4*>(slots + off) = acc;
             if (!GRED && fa.logits_out != nullptr && grow < fa.route.M)
@@ -356,6 +452,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (t == 0) fa.ws_ticket[rank] = 0u;  // ready for the next call
             }
+        }
+    }
+    if constexpr (SPLIT == 2 && !GRED) {
+        // The router scratch overlays the send buffer: wait until the partner
+        // confirms our partials arrived.
+        if (epi && !ptx::mbar_wait_cluster(sent_bar, 0, kWaitNs)) {
+            if (threadIdx.x == 64) atomicAdd(&g_watchdog_trips_fused, 1u);
+            *s_abort = 1;
         }
     }
     ptx::tc_fence_before();

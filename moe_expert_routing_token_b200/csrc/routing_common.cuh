@@ -212,6 +212,16 @@ __device__ __forceinline__ void segment_top8(float v1, float v2, float (&out)[8]
     for (int i = 0; i < 8; ++i) out[i] = a[i];
 }
 
+// The K-th largest (1 <= K <= 8) of a descending list: the minimum of its
+// first K entries (no dynamically indexed array, which would go to local
+// memory).
+__device__ __forceinline__ float kth_of_sorted8(const float (&top)[8], int K) {
+    float t = top[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) t = (i < K) ? fminf(t, top[i]) : t;
+    return t;
+}
+
 // As segment_top8, each lane contributing four values (any order): sort
 // them, merge with the xor-1 partner into a sorted 8, then keep the top 8
 // over the xor-2 and xor-4 partners.

@@ -175,10 +175,7 @@ struct SegRouter {
             // are K distinct kept experts).
             float top[8];
             segment_top8<L>(gsel ? m1 : -INFINITY, gsel ? m2 : -INFINITY, top);
-            tau = top[0];
-#pragma unroll
-            for (int i = 1; i < 8; ++i)
-                if (i == K - 1) tau = top[i];
+            tau = kth_of_sorted8(top, K);
         } else {
             const float my = gsel ? m2 : -INFINITY;
             int r = 0;

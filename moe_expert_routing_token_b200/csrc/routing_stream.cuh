@@ -93,16 +93,6 @@ __device__ __forceinline__ void insert_desc(uint32_t (&kk)[N], int (&ii)[N], uin
     ii[0] = c[0] ? e : ii[0];
 }
 
-// The K-th largest (1 <= K <= 8) of a descending list: the minimum of its
-// first K entries (no dynamically indexed array, which would go to local
-// memory).
-__device__ __forceinline__ float kth_of_sorted8(const float (&top)[8], int K) {
-    float t = top[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) t = (i < K) ? fminf(t, top[i]) : t;
-    return t;
-}
-
 template <typename TIn, int E, int C, int SCORE, bool BIAS, bool APPROX>
 struct StreamCfg {
     static constexpr int L = E / C;                      // lanes per row in phase 1
