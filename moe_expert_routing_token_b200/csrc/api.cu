@@ -164,8 +164,21 @@ int launch_ring(RingKernel kern, size_t smem, int threads, int box_e, int rb, co
     const int64_t nblocks = (a.M + rb - 1) / rb;
     const int64_t cap = (int64_t)sms * per_sm;
     const int grid = (int)(nblocks < cap ? nblocks : cap);
-    kern<<<grid, threads, smem, st>>>(tmap, a, nblocks);
-    err = cudaGetLastError();
+    // Programmatic dependent launch: the block's prologue (barrier set-up,
+    // descriptor prefetch) overlaps the previous kernel in the stream; the
+    // kernel waits for that kernel (griddepcontrol.wait) before it touches any
+    // input or output.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, kern, tmap, a, nblocks);
     if (err != cudaSuccess) return cuda_fail(err, what);
     return MOE_OK;
 }

@@ -125,3 +125,27 @@ def test_close_keys_e160(dtype):
     bias = inputs.random_bias(E, 2e-5, seed=6)
     check("sigmoid", x, bias, 6, True, 8, 3, 1.0)
     check("sigmoid", x, bias, 6, False, 1, 1, 1.0)
+
+
+def test_inputs_written_by_the_previous_kernel():
+    """The streaming kernel starts while the previous kernel in the stream may
+    still run (programmatic dependent launch) and must read its inputs only
+    after that kernel has finished: rewrite the logits in place right before
+    each call and compare with a fresh call on the final data."""
+    import moe_expert_routing_token_b200 as moe
+    M, E, k = 16384, 256, 8
+    dev = "cuda:0"
+    pool = [inputs.random_logits(M, E, 2.0, torch.bfloat16, seed=100 + i).to(dev) for i in range(4)]
+    bias = inputs.random_bias(E, 0.05, seed=9).to(dev)
+    x = torch.empty_like(pool[0])
+    outs = []
+    for rep in range(3):
+        for i in range(4):
+            x.copy_(pool[i])                     # a torch kernel writes the input ...
+            w, ids = moe.biased_grouped_topk(x, bias, k, True, 1, 1, 1.0)  # ... read at once
+            outs.append((i, w, ids))
+    torch.cuda.synchronize()
+    for i, w, ids in outs:
+        w_ref, ids_ref = moe.biased_grouped_topk(pool[i].clone(), bias, k, True, 1, 1, 1.0)
+        torch.cuda.synchronize()
+        assert torch.equal(ids, ids_ref) and torch.equal(w, w_ref)
