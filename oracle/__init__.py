@@ -64,6 +64,9 @@ def _bind(path: str):
     lib.oracle_router_logits.restype = ctypes.c_int
     lib.oracle_router_logits.argtypes = [
         _DBL, _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _DBL]
+    lib.oracle_expert_permutation.restype = ctypes.c_int
+    lib.oracle_expert_permutation.argtypes = [
+        _I32, _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, _I32, _I32, _I32, _I32, _DBL]
     return lib
 
 
@@ -183,3 +186,36 @@ def fused_router_topk(hidden_states, router_weight, correction_bias, topk: int,
     r = biased_grouped_topk(logits, correction_bias, topk, renormalize, num_expert_group,
                             topk_group, routed_scaling_factor, lib=lib)
     return r, logits
+
+
+class Permutation:
+    """Expert-sorted token permutation (all numpy): counts (E,), offsets (E+1,),
+    gather (M*k,), scatter (M*k,), gate (M*k,) float64 or None."""
+
+    def __init__(self, counts, offsets, gather, scatter, gate):
+        self.counts, self.offsets, self.gather, self.scatter, self.gate = counts, offsets, gather, scatter, gate
+
+
+def expert_permutation(topk_ids, num_experts: int, topk_weights=None, lib=None) -> Permutation:
+    """Stable counting sort of the (token, slot) pairs of topk_ids (M, k) by
+    expert id (oracle_expert_permutation)."""
+    if hasattr(topk_ids, "detach"):
+        topk_ids = topk_ids.detach().cpu().numpy()
+    ids = np.ascontiguousarray(np.asarray(topk_ids, dtype=np.int32))
+    if ids.ndim != 2:
+        raise ValueError("topk_ids must be (M, k)")
+    M, k = ids.shape
+    n = M * k
+    w = None if topk_weights is None else as_f64(topk_weights).reshape(-1)
+    counts = np.zeros(num_experts, np.int32)
+    offsets = np.zeros(num_experts + 1, np.int32)
+    gather = np.zeros(n, np.int32)
+    scatter = np.zeros(n, np.int32)
+    gate = None if w is None else np.zeros(n, np.float64)
+    lib = lib or load()
+    rc = lib.oracle_expert_permutation(_ptr(ids, _I32), _ptr(w, _DBL), M, k, int(num_experts),
+                                       _ptr(counts, _I32), _ptr(offsets, _I32), _ptr(gather, _I32),
+                                       _ptr(scatter, _I32), _ptr(gate, _DBL))
+    if rc != 0:
+        raise ValueError("oracle_expert_permutation: invalid arguments (ids outside [0, E)?)")
+    return Permutation(counts, offsets, gather, scatter, gate)

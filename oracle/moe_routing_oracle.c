@@ -254,3 +254,42 @@ int oracle_router_logits(const double* h, const double* w, int64_t M, int K, int
     }
     return ORACLE_OK;
 }
+
+/* ---------------------------------------------------------------------------
+ * oracle_expert_permutation: the expert-sorted token permutation that the
+ * routing page's "Triton Kernels routing" branch hands to the expert runner
+ * ([R] 구조도, 출력 포맷: RoutingData, GatherIndx, ScatterIndx).  The pages give
+ * only the names; the reading taken is a stable counting sort of the M*k
+ * (token, slot) pairs by expert id, pair index i = token*k + slot:
+ *   counts[e]      number of pairs routed to expert e
+ *   offsets[e]     sum of counts[0..e), offsets[E] = M*k
+ *   gather[p]      the pair index at sorted position p (experts ascending,
+ *                  pair index ascending within an expert)
+ *   scatter[i]     the sorted position of pair i (gather[scatter[i]] == i)
+ *   gate[p]        weights[gather[p]] (NULL weights or gate: skipped)
+ * Ids outside [0, E) are rejected.
+ * ------------------------------------------------------------------------- */
+int oracle_expert_permutation(const int32_t* ids, const double* weights, int64_t M, int k, int E,
+                              int32_t* counts, int32_t* offsets, int32_t* gather, int32_t* scatter,
+                              double* gate) {
+    if (M < 0 || k < 1 || E < 1) return ORACLE_BAD_ARGS;
+    const int64_t n = M * (int64_t)k;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        if (ids[i] < 0 || ids[i] >= E) return ORACLE_BAD_ARGS;
+        counts[ids[i]] += 1;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+    if (!cursor) return ORACLE_NO_MEMORY;
+    for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
+    for (int64_t i = 0; i < n; ++i) {       /* pairs in ascending index: stable */
+        const int32_t p = cursor[ids[i]]++;
+        gather[p] = (int32_t)i;
+        scatter[i] = p;
+        if (weights && gate) gate[p] = weights[i];
+    }
+    free(cursor);
+    return ORACLE_OK;
+}

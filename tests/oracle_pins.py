@@ -13,7 +13,10 @@ Pins used:
   with the largest total selection score (unique for distinct values);
 * library cross-checks for the ungrouped cases: scipy's softmax / expit and a
   stable numpy argsort reproduce the scores, ids and weights;
-* the router projection against numpy's float64 matmul and a hand case.
+* the router projection against numpy's float64 matmul and a hand case;
+* the expert permutation against a hand case, and against numpy's stable
+  argsort, bincount and cumsum on random and routed ids (plus its inverse-
+  permutation and stability invariants).
 """
 from __future__ import annotations
 
@@ -215,7 +218,50 @@ def check_library(lib, seed=5) -> list[str]:
     return fails
 
 
-ALL_CHECKS = (check_golden, check_router_golden, check_router_numpy, check_brute, check_library)
+def check_permutation_golden(lib) -> list[str]:
+    doc = json.load(open(os.path.join(GOLDEN, "expert_permutation_small.json")))
+    p = oracle.expert_permutation(np.asarray(doc["topk_ids"], np.int32), doc["num_experts"],
+                                  np.asarray(doc["topk_weights"], np.float64), lib=lib)
+    fails = []
+    for key in ("counts", "offsets", "gather", "scatter"):
+        if getattr(p, key).tolist() != doc[key]:
+            fails.append(f"permutation hand case: {key} {getattr(p, key).tolist()} != {doc[key]}")
+    if p.gate.tolist() != doc["gate"]:
+        fails.append(f"permutation hand case: gate {p.gate.tolist()}")
+    return fails
+
+
+def check_permutation_numpy(lib, seed=13) -> list[str]:
+    """numpy's stable argsort / bincount / cumsum define the same permutation."""
+    rng = np.random.default_rng(seed)
+    fails = []
+    cases = [(rng.integers(0, 16, size=(37, 3)), 16), (rng.integers(0, 3, size=(50, 2)), 8),
+             (np.zeros((9, 4), np.int64), 5), (rng.integers(0, 256, size=(300, 8)), 256)]
+    # ids produced by routing (distinct within a row)
+    x = rng.normal(0, 2, size=(120, 64))
+    cases.append((oracle.topk_softmax(x, 6, True, lib=lib).ids, 64))
+    for n, (ids, E) in enumerate(cases):
+        ids = np.asarray(ids, np.int32)
+        w = rng.random(ids.shape)
+        p = oracle.expert_permutation(ids, E, w, lib=lib)
+        flat = ids.reshape(-1)
+        order = np.argsort(flat, kind="stable")
+        counts = np.bincount(flat, minlength=E)
+        if not np.array_equal(p.gather, order):
+            fails.append(f"permutation case {n}: gather differs from stable argsort")
+        if not np.array_equal(p.counts, counts):
+            fails.append(f"permutation case {n}: counts differ from bincount")
+        if not np.array_equal(p.offsets, np.concatenate([[0], np.cumsum(counts)])):
+            fails.append(f"permutation case {n}: offsets differ from cumsum")
+        if not np.array_equal(p.gather[p.scatter], np.arange(flat.size)):
+            fails.append(f"permutation case {n}: scatter is not the inverse of gather")
+        if not np.array_equal(p.gate, w.reshape(-1)[order]):
+            fails.append(f"permutation case {n}: gate is not the sorted weights")
+    return fails
+
+
+ALL_CHECKS = (check_golden, check_router_golden, check_router_numpy, check_brute, check_library,
+              check_permutation_golden, check_permutation_numpy)
 
 
 def run_all(lib) -> list[str]:

@@ -38,6 +38,11 @@ MUTANTS = {
     "ascending_order": ("if (a->value > b->value) return -1;\n    if (a->value < b->value) return 1;",
                         "if (a->value > b->value) return 1;\n    if (a->value < b->value) return -1;"),
     "group_max_is_min": ("if (s[first + j] > m) m = s[first + j];", "if (s[first + j] < m) m = s[first + j];"),
+    "perm_unstable": ("for (int64_t i = 0; i < n; ++i) {       /* pairs in ascending index: stable */",
+                      "for (int64_t i = n - 1; i >= 0; --i) {       /* reversed: not stable */"),
+    "perm_inclusive_offsets": ("for (int e = 0; e < E; ++e) cursor[e] = offsets[e];",
+                               "for (int e = 0; e < E; ++e) cursor[e] = offsets[e + 1] - 1;"),
+    "perm_scatter_is_gather": ("        scatter[i] = p;\n", "        scatter[p] = (int32_t)i;\n"),
 }
 
 
