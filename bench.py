@@ -46,7 +46,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=480)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="sigmoid",
-                    choices=["sigmoid", "biased", "grouped", "softmax", "fused"])
+                    choices=["sigmoid", "biased", "grouped", "softmax", "fused", "permute"])
     ap.add_argument("--M", type=int, default=None, help="tokens per step (default: workload's)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -55,7 +55,8 @@ def parse_args():
     return ap.parse_args()
 
 
-DEFAULT_M = {"sigmoid": 16384, "biased": 4096, "grouped": 16384, "softmax": 64, "fused": 8192}
+DEFAULT_M = {"sigmoid": 16384, "biased": 4096, "grouped": 16384, "softmax": 64, "fused": 8192, "permute": 16384}
+PERM_K, PERM_E = 8, 256  # the permutation step after the sigmoid workload's routing
 
 
 def workload_desc(name: str, M: int) -> dict:
@@ -504,8 +505,212 @@ def e2e_measure(name, M, sp, d, dev, stream, world, args):
             "d2h_bytes_per_step": hw.numel() * 4 + hi.numel() * 4, "steps": steps}
 
 
+# ---------------------------------------------------------------------------
+# The expert permutation after routing (moe_expert_permutation)
+PERM_METRIC = "permuted tokens/s & us/call (expert-sorted permutation of (M, k=8) ids, E=256); % of HBM roofline"
+
+
+def perm_bytes(M: int) -> int:
+    """Bytes a permutation call must move: ids and weights in; gather, scatter
+    and gate out; counts and offsets."""
+    n = M * PERM_K
+    return n * 4 * 5 + (2 * PERM_E + 1) * 4
+
+
+def perm_desc(M: int) -> dict:
+    return {"M": M, "k": PERM_K, "E": PERM_E,
+            "workload": (f"expert-sorted permutation of a routing result: topk_ids (M={M}, k={PERM_K}) int32 "
+                         f"(k distinct uniform experts of E={PERM_E} per token), fp32 weights -> counts, "
+                         f"offsets, gather, scatter, gate")}
+
+
+def time_perm_oracle(M: int, seconds: float) -> dict:
+    import oracle
+    from moe_expert_routing_token_b200 import inputs
+    ids, w = inputs.routed_ids(M, PERM_K, PERM_E, seed=4242)
+    ids_np, w_np = ids.numpy(), w.numpy()
+    oracle.expert_permutation(ids_np[:8], PERM_E, w_np[:8])
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.expert_permutation(ids_np, PERM_E, w_np)
+        n += M
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens ({n // M} x {M}-token batches), single-threaded C oracle, {el:.1f} s"}
+
+
+def run_permute(args):
+    import torch
+    import torch.distributed as dist
+
+    from moe_expert_routing_token_b200 import build, inputs, routing
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        M = args.M or DEFAULT_M["permute"]
+        base = time_perm_oracle(M, min(args.cpu_seconds, 10.0))
+        line = {"impl": "reference", "metric": PERM_METRIC, "value": base["value"], "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": M / base["value"] * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "int32", "data": "synthetic", "config": perm_desc(M),
+                "cpu_baseline": base,
+                "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device; the routing library has no CPU path")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    lib = routing.lib()
+    M = args.M or DEFAULT_M["permute"]
+    n = M * PERM_K
+    ids_h, w_h = inputs.routed_ids(M, PERM_K, PERM_E, seed=rank_seed("sigmoid", M, rank))
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    sptr = stream.cuda_stream
+    per_set = perm_bytes(M)
+    pool = max(2, min(256, -(-4 * L2_BYTES // per_set)))
+    ids = [ids_h.to(dev) for _ in range(pool)]
+    wts = [w_h.to(dev) for _ in range(pool)]
+    outs = [[torch.empty(PERM_E, dtype=torch.int32, device=dev), torch.empty(PERM_E + 1, dtype=torch.int32, device=dev),
+             torch.empty(n, dtype=torch.int32, device=dev), torch.empty(n, dtype=torch.int32, device=dev),
+             torch.empty(n, dtype=torch.float32, device=dev)] for _ in range(pool)]
+    wsb = routing.expert_permutation_workspace_size(M, PERM_K, PERM_E)
+    wsp = [torch.empty(max(1, wsb), dtype=torch.uint8, device=dev) for _ in range(pool)]
+
+    def call(i: int, src_ids=None, src_w=None, out=None, ws=None):
+        j = i % pool
+        o = out if out is not None else outs[j]
+        st = lib.moe_expert_permutation((src_ids if src_ids is not None else ids[j]).data_ptr(),
+                                        (src_w if src_w is not None else wts[j]).data_ptr(), M, PERM_K, PERM_E,
+                                        o[0].data_ptr(), o[1].data_ptr(), o[2].data_ptr(), o[3].data_ptr(),
+                                        o[4].data_ptr(), (ws if ws is not None else wsp[j]).data_ptr(), wsb, sptr)
+        if st != 0:
+            raise RuntimeError(lib.moe_last_error().decode())
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize()
+
+    def capture(nsteps: int):
+        if nsteps == 0:
+            return None
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(nsteps):
+                call(i)
+        return g
+
+    with torch.cuda.stream(stream):
+        g_pool = capture(pool)
+        g_rem = capture(args.steps % pool)
+        g_warm_rem = capture(args.warmup % pool)
+
+    def run_steps(nst: int, rem_graph):
+        for _ in range(nst // pool):
+            g_pool.replay()
+        if rem_graph is not None:
+            rem_graph.replay()
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    run_steps(args.warmup, g_warm_rem)
+    t_soak = time.time()
+    while not args.no_soak and time.time() - t_soak < 1.0:
+        g_pool.replay()
+        torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    run_steps(args.steps, g_rem)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = job_elapsed_ms(start.elapsed_time(stop), world, dev)
+    clocks = sampler.stop() if sampler else None
+    value = job_tokens_per_s(M, args.steps, world, ms)
+    us_per_call = ms * 1e3 / args.steps
+
+    e2e = None
+    if not args.no_e2e:
+        # host buffers in, permutation out, every step
+        h_ids = ids_h.pin_memory()
+        h_w = w_h.pin_memory()
+        h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs[0]]
+        d_ids, d_w = ids[0], wts[0]
+        steps = 200
+
+        def step():
+            d_ids.copy_(h_ids, non_blocking=True)
+            d_w.copy_(h_w, non_blocking=True)
+            call(0, d_ids, d_w, outs[0], wsp[0])
+            for h, d in zip(h_out, outs[0]):
+                h.copy_(d, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                step()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                step()
+            b.record(stream)
+            torch.cuda.synchronize()
+        ems = job_elapsed_ms(a.elapsed_time(b), world, dev)
+        e2e = {"value": job_tokens_per_s(M, steps, world, ems), "unit": "tokens/s",
+               "h2d_bytes_per_step": n * 8, "d2h_bytes_per_step": sum(t.numel() * 4 for t in h_out),
+               "steps": steps}
+
+    peaks = measured_peaks()
+    achieved = per_set / (us_per_call * 1e-6) / 1e9
+    line = {"metric": PERM_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "us_per_call": us_per_call, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int32", "data": "synthetic",
+            "config": dict(perm_desc(M), parallelism=f"dp{world} (rows sharded, no collective)",
+                           l2=f"rotating pool of {pool} sets, {pool * per_set / 2**20:.0f} MiB > 126 MiB L2",
+                           timing="CUDA graphs of the C-ABI calls, CUDA events on the launch stream"),
+            "gpu_launches": 3 * args.steps, "clocks": clocks,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_launch": per_set,
+                         "peak_source": f"{peaks['source']} HBM copy"},
+            "e2e": e2e}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = time_perm_oracle(M, args.cpu_seconds)
+    if world > 1:
+        del g_pool, g_rem, g_warm_rem
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.workload == "permute":
+        return run_permute(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -235,6 +235,38 @@ MOE_API int moe_fused_router_topk_noalloc(const void* hidden_states, const void*
                                           float routed_scaling_factor, float* topk_weights,
                                           int32_t* topk_ids, float* logits_out, void* stream);
 
+/*
+ * moe_expert_permutation - the expert-sorted token permutation that follows
+ * routing: the routing page's "Triton Kernels routing" branch hands the expert
+ * runner RoutingData, GatherIndx and ScatterIndx (structure diagram 구조도 and
+ * output format 출력 포맷: TRITON_KERNEL).  The page shows no body; this call
+ * computes a stable counting sort of the M*k (token, slot) pairs of
+ * topk_ids by expert id, with pair index i = token*k + slot.
+ *
+ *   topk_ids       int32 (M, k) row-major, device
+ *   topk_weights   fp32 (M, k) or NULL (then gate_scal must be NULL too)
+ *   expert_counts  int32 (E): pairs routed to each expert
+ *   expert_offsets int32 (E + 1): exclusive prefix of the counts;
+ *                  expert_offsets[E] = number of pairs with an id in [0, E)
+ *   gather_indx    int32 (M*k): pair index at each sorted position (experts
+ *                  ascending, pair index ascending within an expert); only
+ *                  the first expert_offsets[E] entries are written
+ *   scatter_indx   int32 (M*k): sorted position of each pair, -1 for a pair
+ *                  whose id lies outside [0, E) (such pairs are skipped)
+ *   gate_scal      fp32 (M*k) or NULL: topk_weights in sorted order
+ *   workspace      device scratch of moe_expert_permutation_workspace_size()
+ *                  bytes (no initial contents needed; owned by the caller, not
+ *                  shared between calls that may run concurrently)
+ * Deterministic: the same inputs give the same outputs bit for bit.
+ * Limits: E <= 1024 and M*k < 2^31 (else MOE_ERR_UNSUPPORTED).  M = 0
+ * writes zero counts and offsets.  Asynchronous on `stream`; no allocation.
+ */
+MOE_API size_t moe_expert_permutation_workspace_size(int64_t M, int32_t k, int32_t E);
+MOE_API int moe_expert_permutation(const int32_t* topk_ids, const float* topk_weights, int64_t M, int32_t k,
+                                   int32_t E, int32_t* expert_counts, int32_t* expert_offsets,
+                                   int32_t* gather_indx, int32_t* scatter_indx, float* gate_scal,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -11,6 +11,8 @@ from .routing import (  # noqa: F401
     MOE_WEIGHT_K_BY_E,
     RoutingError,
     biased_grouped_topk,
+    expert_permutation,
+    expert_permutation_workspace_size,
     fused_router_topk,
     fused_router_workspace_size,
     grouped_topk,
@@ -21,5 +23,6 @@ from .routing import (  # noqa: F401
 
 __all__ = [
     "topk_softmax", "grouped_topk", "biased_grouped_topk", "fused_router_topk",
-    "fused_router_workspace_size", "lib", "RoutingError", "watchdog_trips",
+    "fused_router_workspace_size", "lib", "RoutingError", "watchdog_trips", "expert_permutation",
+    "expert_permutation_workspace_size",
 ]

@@ -105,3 +105,14 @@ def random_logits(M: int, E: int, std: float, dtype: torch.dtype, seed: int) -> 
 def random_bias(E: int, std: float, seed: int) -> torch.Tensor:
     gen = torch.Generator().manual_seed(int(seed))
     return _normal(gen, (E,), std, torch.float32)
+
+
+def routed_ids(M: int, k: int, E: int, seed: int):
+    """A routing result's shape for the permutation step: per token k distinct
+    experts drawn uniformly (ids int32 (M, k)) and positive weights summing to
+    one per token (fp32 (M, k)).  Balanced routers (the correction bias exists
+    to balance load) spread tokens over experts about uniformly."""
+    gen = torch.Generator().manual_seed(int(seed))
+    ids = torch.argsort(torch.rand(M, E, generator=gen), dim=1)[:, :k].to(torch.int32).contiguous()
+    w = torch.rand(M, k, generator=gen) + 0.05
+    return ids, (w / w.sum(dim=1, keepdim=True)).to(torch.float32)

@@ -46,6 +46,9 @@ SIGNATURES = {
                                              _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_fused_router_topk_noalloc": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32,
                                                      _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
+    "moe_expert_permutation_workspace_size": (_sz, [_i64, _i32, _i32]),
+    "moe_expert_permutation": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                              _vp]),
 }
 
 
@@ -218,3 +221,41 @@ def fused_router_topk(hidden_states: torch.Tensor, router_weight: torch.Tensor, 
                                      need if wsp else 0, _stream(dev))
     _check(st, "moe_fused_router_topk")
     return (w, ids, logits) if return_logits else (w, ids)
+
+
+def expert_permutation_workspace_size(M: int, k: int, E: int) -> int:
+    n = lib().moe_expert_permutation_workspace_size(int(M), int(k), int(E))
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError(f"expert_permutation_workspace_size: bad sizes M={M} k={k} E={E}")
+    return n
+
+
+def expert_permutation(topk_ids: torch.Tensor, num_experts: int, topk_weights=None, workspace=None):
+    """Expert-sorted permutation of a routing result (see
+    moe_expert_permutation in include/moe_routing.h).  Returns
+    (expert_counts, expert_offsets, gather_indx, scatter_indx, gate_scal);
+    gate_scal is None when topk_weights is None."""
+    _cuda_2d(topk_ids, "topk_ids")
+    if topk_ids.dtype != torch.int32:
+        raise ValueError("topk_ids must be int32")
+    M, k = topk_ids.shape
+    dev = topk_ids.device
+    n = M * k
+    if topk_weights is not None:
+        _cuda_2d(topk_weights, "topk_weights")
+        if topk_weights.dtype != torch.float32 or tuple(topk_weights.shape) != (M, k):
+            raise ValueError("topk_weights must be fp32 with the shape of topk_ids")
+    need = expert_permutation_workspace_size(M, k, num_experts)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    counts = torch.empty(num_experts, dtype=torch.int32, device=dev)
+    offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    gather = torch.empty(n, dtype=torch.int32, device=dev)
+    scatter = torch.empty(n, dtype=torch.int32, device=dev)
+    gate = None if topk_weights is None else torch.empty(n, dtype=torch.float32, device=dev)
+    _check(lib().moe_expert_permutation(
+        topk_ids.data_ptr(), None if topk_weights is None else topk_weights.data_ptr(), M, k, int(num_experts),
+        counts.data_ptr(), offsets.data_ptr(), gather.data_ptr(), scatter.data_ptr(),
+        None if gate is None else gate.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(dev)),
+        "moe_expert_permutation")
+    return counts, offsets, gather, scatter, gate

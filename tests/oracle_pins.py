@@ -257,6 +257,16 @@ def check_permutation_numpy(lib, seed=13) -> list[str]:
             fails.append(f"permutation case {n}: scatter is not the inverse of gather")
         if not np.array_equal(p.gate, w.reshape(-1)[order]):
             fails.append(f"permutation case {n}: gate is not the sorted weights")
+    # ids outside [0, E) are skipped: the valid pairs keep their stable order
+    ids = rng.integers(-3, 12, size=(40, 3)).astype(np.int32)
+    p = oracle.expert_permutation(ids, 10, lib=lib)
+    flat = ids.reshape(-1)
+    ok = (flat >= 0) & (flat < 10)
+    order = np.nonzero(ok)[0][np.argsort(flat[ok], kind="stable")]
+    if not np.array_equal(p.gather[: ok.sum()], order) or p.offsets[-1] != ok.sum():
+        fails.append("permutation with invalid ids: valid pairs misplaced")
+    if not np.all(p.scatter[~ok] == -1) or not np.array_equal(p.scatter[order], np.arange(ok.sum())):
+        fails.append("permutation with invalid ids: scatter wrong")
     return fails
 
 

@@ -92,3 +92,17 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(4, 8)
     with pytest.raises(ValueError):
         moe.topk_softmax(x, 2, True)
+
+
+def test_expert_permutation_validation(lib):
+    ws = lib.moe_expert_permutation_workspace_size(16384, 8, 256)
+    assert ws == 128 * 256 * 4                       # one int32 per (1024-pair tile, expert)
+    assert lib.moe_expert_permutation_workspace_size(10, 8, 2048) == ctypes.c_size_t(-1).value
+    # (ids, weights, M, k, E, counts, offsets, gather, scatter, gate, workspace, bytes, stream)
+    assert lib.moe_expert_permutation(P, None, 4, 0, 16, P, P, P, P, None, P, 4096, None) == 1   # k < 1
+    assert lib.moe_expert_permutation(P, None, 4, 2, 2048, P, P, P, P, None, P, 4096, None) == 2  # E > 1024
+    assert b"E=2048" in lib.moe_last_error()
+    assert lib.moe_expert_permutation(P, P, 4, 2, 16, P, P, P, P, None, P, 4096, None) == 1     # gate missing
+    assert lib.moe_expert_permutation(P, None, 4, 2, 16, P, P, P, P, None, P, 3, None) == 1     # workspace short
+    assert b"workspace" in lib.moe_last_error()
+    assert lib.moe_expert_permutation(P, None, 4, 2, 16, None, P, P, P, None, P, 4096, None) == 1  # no counts
