@@ -198,7 +198,8 @@ class Permutation:
 
 def expert_permutation(topk_ids, num_experts: int, topk_weights=None, lib=None) -> Permutation:
     """Stable counting sort of the (token, slot) pairs of topk_ids (M, k) by
-    expert id (oracle_expert_permutation)."""
+    expert id (oracle_expert_permutation); pairs with an id outside [0, E) are
+    skipped (scatter -1, gather holds offsets[E] entries)."""
     if hasattr(topk_ids, "detach"):
         topk_ids = topk_ids.detach().cpu().numpy()
     ids = np.ascontiguousarray(np.asarray(topk_ids, dtype=np.int32))
@@ -217,5 +218,5 @@ def expert_permutation(topk_ids, num_experts: int, topk_weights=None, lib=None) 
                                        _ptr(counts, _I32), _ptr(offsets, _I32), _ptr(gather, _I32),
                                        _ptr(scatter, _I32), _ptr(gate, _DBL))
     if rc != 0:
-        raise ValueError("oracle_expert_permutation: invalid arguments (ids outside [0, E)?)")
+        raise ValueError("oracle_expert_permutation: invalid arguments")
     return Permutation(counts, offsets, gather, scatter, gate)

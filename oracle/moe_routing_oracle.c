@@ -267,7 +267,8 @@ int oracle_router_logits(const double* h, const double* w, int64_t M, int K, int
  *                  pair index ascending within an expert)
  *   scatter[i]     the sorted position of pair i (gather[scatter[i]] == i)
  *   gate[p]        weights[gather[p]] (NULL weights or gate: skipped)
- * Ids outside [0, E) are rejected.
+ * A pair whose id lies outside [0, E) is skipped: not counted, not placed,
+ * scatter = -1 (offsets[E] is then the number of placed pairs).
  * ------------------------------------------------------------------------- */
 int oracle_expert_permutation(const int32_t* ids, const double* weights, int64_t M, int k, int E,
                               int32_t* counts, int32_t* offsets, int32_t* gather, int32_t* scatter,
@@ -275,16 +276,18 @@ int oracle_expert_permutation(const int32_t* ids, const double* weights, int64_t
     if (M < 0 || k < 1 || E < 1) return ORACLE_BAD_ARGS;
     const int64_t n = M * (int64_t)k;
     for (int e = 0; e < E; ++e) counts[e] = 0;
-    for (int64_t i = 0; i < n; ++i) {
-        if (ids[i] < 0 || ids[i] >= E) return ORACLE_BAD_ARGS;
-        counts[ids[i]] += 1;
-    }
+    for (int64_t i = 0; i < n; ++i)
+        if (ids[i] >= 0 && ids[i] < E) counts[ids[i]] += 1;
     offsets[0] = 0;
     for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
     int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
     if (!cursor) return ORACLE_NO_MEMORY;
     for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
     for (int64_t i = 0; i < n; ++i) {       /* pairs in ascending index: stable */
+        if (ids[i] < 0 || ids[i] >= E) {
+            scatter[i] = -1;
+            continue;
+        }
         const int32_t p = cursor[ids[i]]++;
         gather[p] = (int32_t)i;
         scatter[i] = p;
