@@ -64,6 +64,11 @@ def _bind(path: str):
     lib.oracle_router_logits.restype = ctypes.c_int
     lib.oracle_router_logits.argtypes = [
         _DBL, _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _DBL]
+    lib.oracle_fill_shared_slot.restype = ctypes.c_int
+    lib.oracle_fill_shared_slot.argtypes = [_DBL, _I32, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            _I32, ctypes.c_double]
+    lib.oracle_sort_by_id.restype = ctypes.c_int
+    lib.oracle_sort_by_id.argtypes = [_DBL, _I32, ctypes.c_int64, ctypes.c_int]
     lib.oracle_expert_permutation.restype = ctypes.c_int
     lib.oracle_expert_permutation.argtypes = [
         _I32, _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, _I32, _I32, _I32, _I32, _DBL]
@@ -220,3 +225,35 @@ def expert_permutation(topk_ids, num_experts: int, topk_weights=None, lib=None) 
     if rc != 0:
         raise ValueError("oracle_expert_permutation: invalid arguments")
     return Permutation(counts, offsets, gather, scatter, gate)
+
+
+def fill_shared_slot(topk_weights, topk_ids, num_experts: int, num_shared: int, picks,
+                     routed_scaling_factor=None, lib=None):
+    """[R] §6 on a routing result: last slot -> shared expert E + pick, weight
+    -> sum of the other weights / routed_scaling_factor (unchanged if None).
+    Returns new (weights float64, ids int32) arrays."""
+    w = as_f64(topk_weights).copy()
+    ids = np.ascontiguousarray(np.asarray(topk_ids if not hasattr(topk_ids, "detach") else topk_ids.cpu().numpy(),
+                                          dtype=np.int32)).copy()
+    pk = np.ascontiguousarray(np.asarray(picks if not hasattr(picks, "detach") else picks.cpu().numpy(),
+                                         dtype=np.int32))
+    M, k = ids.shape
+    rsf = 0.0 if routed_scaling_factor is None else float(routed_scaling_factor)
+    lib = lib or load()
+    rc = lib.oracle_fill_shared_slot(_ptr(w, _DBL), _ptr(ids, _I32), M, k, int(num_experts), int(num_shared),
+                                     _ptr(pk, _I32), rsf)
+    if rc != 0:
+        raise ValueError("oracle_fill_shared_slot: invalid arguments")
+    return w, ids
+
+
+def sort_by_id(topk_weights, topk_ids, lib=None):
+    """Each row's (weight, id) pairs in ascending id, stable.  Returns new arrays."""
+    w = as_f64(topk_weights).copy()
+    ids = np.ascontiguousarray(np.asarray(topk_ids if not hasattr(topk_ids, "detach") else topk_ids.cpu().numpy(),
+                                          dtype=np.int32)).copy()
+    M, k = ids.shape
+    lib = lib or load()
+    if lib.oracle_sort_by_id(_ptr(w, _DBL), _ptr(ids, _I32), M, k) != 0:
+        raise ValueError("oracle_sort_by_id: invalid arguments")
+    return w, ids

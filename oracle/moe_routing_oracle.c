@@ -11,6 +11,8 @@
  * exp() and qsort().  There is deliberately no blocking, fusion or cleverness.
  *
  * Sources (pages on SGLang MoE routing; cited by page title and section):
+ *   [M] "MiniMax-M3 모델을 위한 FP8 Attention GEMM 최적화 및 성능 개선"
+ *       코드 분석 §1 minimax_decode_topk - ascending (sorted) id output
  *   [R] "[SGLang] MoE 라우팅: 토큰에서 전문가로의 배분 알고리즘"
  *       (SGLang MoE routing: token-to-expert algorithms)
  *       §2 기본 softmax Top-K     - softmax scores, top-k, renormalise
@@ -22,6 +24,7 @@
  *                                   biased scores in the group
  *       §5 Fused MoE Router       - logits = hidden_states x router weight in
  *                                   fp32 accumulation, routing on the result
+ *       §6 공유 전문가 슬롯 할당       - the last slot goes to a shared expert
  *   [A] "[sglang] SGLang MoE 라우팅 최적화: AMD GPU에서 aiter.biased_grouped_topk 활용"
  *       코드 분석 (After)           - sigmoid + correction_bias routing expressed
  *                                   as biased grouped top-k with
@@ -294,5 +297,54 @@ int oracle_expert_permutation(const int32_t* ids, const double* weights, int64_t
         if (weights && gate) gate[p] = weights[i];
     }
     free(cursor);
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * oracle_fill_shared_slot: the shared-expert slot of [R] §6 (공유 전문가 슬롯
+ * 할당) on a finished routing result (weights, ids: M x k, in place).  The
+ * last slot of every row gets the shared expert E + pick[i] (pick[i] in
+ * [0, num_shared): the random draw, passed in); when rsf != 0 its weight
+ * becomes the sum of the row's other k-1 weights divided by rsf (rsf == 0:
+ * "routed_scaling_factor is None", the weight is left as it is).
+ * ------------------------------------------------------------------------- */
+int oracle_fill_shared_slot(double* weights, int32_t* ids, int64_t M, int k, int E, int num_shared,
+                            const int32_t* pick, double rsf) {
+    if (M < 0 || k < 1 || E < 1 || num_shared < 1) return ORACLE_BAD_ARGS;
+    for (int64_t i = 0; i < M; ++i) {
+        if (pick[i] < 0 || pick[i] >= num_shared) return ORACLE_BAD_ARGS;
+        ids[i * (int64_t)k + (k - 1)] = E + pick[i];
+        if (rsf != 0.0) {
+            double sum = 0.0;
+            for (int j = 0; j < k - 1; ++j) sum += weights[i * (int64_t)k + j];
+            weights[i * (int64_t)k + (k - 1)] = sum / rsf;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * oracle_sort_by_id: reorder every row's k (weight, id) pairs by ascending
+ * id, equal ids keeping their order - the ascending expert/block-id output
+ * that [M] 코드 분석 §1 (minimax_decode_topk) produces with a warp rank sort.
+ * ------------------------------------------------------------------------- */
+int oracle_sort_by_id(double* weights, int32_t* ids, int64_t M, int k) {
+    if (M < 0 || k < 1) return ORACLE_BAD_ARGS;
+    for (int64_t i = 0; i < M; ++i) {
+        int32_t* id = ids + i * (int64_t)k;
+        double* w = weights + i * (int64_t)k;
+        for (int a = 1; a < k; ++a) {          /* insertion sort: stable */
+            const int32_t ka = id[a];
+            const double wa = w[a];
+            int b = a - 1;
+            while (b >= 0 && id[b] > ka) {
+                id[b + 1] = id[b];
+                w[b + 1] = w[b];
+                --b;
+            }
+            id[b + 1] = ka;
+            w[b + 1] = wa;
+        }
+    }
     return ORACLE_OK;
 }

@@ -270,8 +270,37 @@ def check_permutation_numpy(lib, seed=13) -> list[str]:
     return fails
 
 
+def check_postprocess(lib) -> list[str]:
+    """Shared-expert slot and ascending-id order: hand cases and invariants."""
+    doc = json.load(open(os.path.join(GOLDEN, "postprocess_small.json")))
+    fails = []
+    sh = doc["shared"]
+    w, ids = oracle.fill_shared_slot(np.asarray(sh["weights"]), np.asarray(sh["ids"]), sh["num_experts"],
+                                     sh["num_shared"], np.asarray(sh["pick"]), sh["routed_scaling_factor"], lib=lib)
+    if ids.tolist() != sh["out_ids"] or not np.allclose(w, sh["out_weights"], rtol=0, atol=1e-15):
+        fails.append(f"shared slot hand case: {ids.tolist()} {w.tolist()}")
+    w, ids = oracle.fill_shared_slot(np.asarray(sh["weights"]), np.asarray(sh["ids"]), sh["num_experts"],
+                                     sh["num_shared"], np.asarray(sh["pick"]), None, lib=lib)
+    if ids.tolist() != sh["out_ids"] or w.tolist() != sh["out_weights_no_scale"]:
+        fails.append("shared slot without a scaling factor changed the weight")
+    so = doc["sort"]
+    w, ids = oracle.sort_by_id(np.asarray(so["weights"]), np.asarray(so["ids"]), lib=lib)
+    if ids.tolist() != so["out_ids"] or w.tolist() != so["out_weights"]:
+        fails.append(f"ascending-id hand case: {ids.tolist()} {w.tolist()}")
+    # invariants on random rows: a stable sort by id is numpy's stable argsort
+    rng = np.random.default_rng(17)
+    ids0 = rng.integers(0, 6, size=(64, 7)).astype(np.int32)
+    w0 = rng.random((64, 7))
+    w, ids = oracle.sort_by_id(w0, ids0, lib=lib)
+    order = np.argsort(ids0, axis=1, kind="stable")
+    if not np.array_equal(ids, np.take_along_axis(ids0, order, 1)) or \
+            not np.array_equal(w, np.take_along_axis(w0, order, 1)):
+        fails.append("ascending-id order differs from a stable argsort")
+    return fails
+
+
 ALL_CHECKS = (check_golden, check_router_golden, check_router_numpy, check_brute, check_library,
-              check_permutation_golden, check_permutation_numpy)
+              check_permutation_golden, check_permutation_numpy, check_postprocess)
 
 
 def run_all(lib) -> list[str]:

@@ -43,6 +43,10 @@ MUTANTS = {
     "perm_inclusive_offsets": ("for (int e = 0; e < E; ++e) cursor[e] = offsets[e];",
                                "for (int e = 0; e < E; ++e) cursor[e] = offsets[e + 1] - 1;"),
     "perm_scatter_is_gather": ("        scatter[i] = p;\n", "        scatter[p] = (int32_t)i;\n"),
+    "shared_weight_times_rsf": ("weights[i * (int64_t)k + (k - 1)] = sum / rsf;",
+                                "weights[i * (int64_t)k + (k - 1)] = sum * rsf;"),
+    "shared_id_offset": ("ids[i * (int64_t)k + (k - 1)] = E + pick[i];", "ids[i * (int64_t)k + (k - 1)] = pick[i];"),
+    "sort_unstable": ("while (b >= 0 && id[b] > ka) {", "while (b >= 0 && id[b] >= ka) {"),
 }
 
 
