@@ -267,6 +267,31 @@ MOE_API int moe_expert_permutation(const int32_t* topk_ids, const float* topk_we
                                    int32_t* gather_indx, int32_t* scatter_indx, float* gate_scal,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * moe_fill_shared_expert_slot - the shared-expert slot of the routing page
+ * (§6 공유 전문가 슬롯 할당), applied in place to a finished routing result.
+ *
+ *   topk_weights, topk_ids  fp32 / int32 (M, k), device, row-major (in place)
+ *   shared_pick    int32 (M,), device: the random draw per token, each value
+ *                  in [0, num_shared) (the page uses torch.randint); values
+ *                  outside that range are not checked
+ *   routed_scaling_factor   0 = "None": the last slot's weight is left as it
+ *                  is; otherwise it becomes (sum of the row's other k-1
+ *                  weights, fp32 in slot order) / routed_scaling_factor
+ * The last slot's id becomes E + shared_pick[row].  k <= 32; M = 0 is a no-op.
+ */
+MOE_API int moe_fill_shared_expert_slot(float* topk_weights, int32_t* topk_ids, int64_t M, int32_t k, int32_t E,
+                                        int32_t num_shared, const int32_t* shared_pick,
+                                        float routed_scaling_factor, void* stream);
+
+/*
+ * moe_sort_topk_by_id - reorder every row's k (weight, id) pairs by ascending
+ * id in place, equal ids keeping their order: the ascending id output that the
+ * MiniMax-M3 page's minimax_decode_topk produces with a warp-wise rank sort
+ * (코드 분석 §1).  k <= 32; M = 0 is a no-op.
+ */
+MOE_API int moe_sort_topk_by_id(float* topk_weights, int32_t* topk_ids, int64_t M, int32_t k, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,10 +13,12 @@ from .routing import (  # noqa: F401
     biased_grouped_topk,
     expert_permutation,
     expert_permutation_workspace_size,
+    fill_shared_expert_slot,
     fused_router_topk,
     fused_router_workspace_size,
     grouped_topk,
     lib,
+    sort_topk_by_id,
     topk_softmax,
     watchdog_trips,
 )
@@ -24,5 +26,5 @@ from .routing import (  # noqa: F401
 __all__ = [
     "topk_softmax", "grouped_topk", "biased_grouped_topk", "fused_router_topk",
     "fused_router_workspace_size", "lib", "RoutingError", "watchdog_trips", "expert_permutation",
-    "expert_permutation_workspace_size",
+    "expert_permutation_workspace_size", "fill_shared_expert_slot", "sort_topk_by_id",
 ]

@@ -47,6 +47,8 @@ SIGNATURES = {
     "moe_fused_router_topk_noalloc": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32,
                                                      _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
     "moe_expert_permutation_workspace_size": (_sz, [_i64, _i32, _i32]),
+    "moe_fill_shared_expert_slot": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _i32, _vp, _f32, _vp]),
+    "moe_sort_topk_by_id": (ctypes.c_int, [_vp, _vp, _i64, _i32, _vp]),
     "moe_expert_permutation": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                               _vp]),
 }
@@ -259,3 +261,38 @@ def expert_permutation(topk_ids: torch.Tensor, num_experts: int, topk_weights=No
         None if gate is None else gate.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(dev)),
         "moe_expert_permutation")
     return counts, offsets, gather, scatter, gate
+
+
+def _result_pair(topk_weights: torch.Tensor, topk_ids: torch.Tensor):
+    _cuda_2d(topk_weights, "topk_weights")
+    _cuda_2d(topk_ids, "topk_ids")
+    if topk_weights.dtype != torch.float32 or topk_ids.dtype != torch.int32 or \
+            topk_weights.shape != topk_ids.shape:
+        raise ValueError("topk_weights must be fp32 and topk_ids int32 of the same (M, k) shape")
+    return topk_ids.shape
+
+
+def fill_shared_expert_slot(topk_weights: torch.Tensor, topk_ids: torch.Tensor, num_experts: int,
+                            num_shared: int, shared_pick: torch.Tensor, routed_scaling_factor=None):
+    """In place: the last slot of each row -> shared expert num_experts +
+    shared_pick[row]; its weight -> sum of the other weights /
+    routed_scaling_factor (unchanged when it is None)."""
+    M, k = _result_pair(topk_weights, topk_ids)
+    if not shared_pick.is_cuda or shared_pick.dtype != torch.int32 or shared_pick.numel() != M or \
+            not shared_pick.is_contiguous():
+        raise ValueError("shared_pick must be a contiguous CUDA int32 tensor of M values")
+    rsf = 0.0 if routed_scaling_factor is None else float(routed_scaling_factor)
+    if routed_scaling_factor is not None and rsf == 0.0:
+        raise ValueError("routed_scaling_factor 0 is reserved for None")
+    _check(lib().moe_fill_shared_expert_slot(topk_weights.data_ptr(), topk_ids.data_ptr(), M, k, int(num_experts),
+                                             int(num_shared), shared_pick.data_ptr(), rsf,
+                                             _stream(topk_ids.device)), "moe_fill_shared_expert_slot")
+    return topk_weights, topk_ids
+
+
+def sort_topk_by_id(topk_weights: torch.Tensor, topk_ids: torch.Tensor):
+    """In place: each row's (weight, id) pairs in ascending id (stable)."""
+    M, k = _result_pair(topk_weights, topk_ids)
+    _check(lib().moe_sort_topk_by_id(topk_weights.data_ptr(), topk_ids.data_ptr(), M, k,
+                                     _stream(topk_ids.device)), "moe_sort_topk_by_id")
+    return topk_weights, topk_ids

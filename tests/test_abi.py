@@ -106,3 +106,16 @@ def test_expert_permutation_validation(lib):
     assert lib.moe_expert_permutation(P, None, 4, 2, 16, P, P, P, P, None, P, 3, None) == 1     # workspace short
     assert b"workspace" in lib.moe_last_error()
     assert lib.moe_expert_permutation(P, None, 4, 2, 16, None, P, P, P, None, P, 4096, None) == 1  # no counts
+
+
+def test_postprocess_validation(lib):
+    # (weights, ids, M, k, E, num_shared, pick, rsf, stream)
+    assert lib.moe_fill_shared_expert_slot(P, P, 4, 0, 256, 1, P, 2.5, None) == 1       # k < 1
+    assert lib.moe_fill_shared_expert_slot(P, P, 4, 33, 256, 1, P, 2.5, None) == 2      # k > 32
+    assert lib.moe_fill_shared_expert_slot(P, P, 4, 9, 256, 0, P, 2.5, None) == 1       # no shared expert
+    assert lib.moe_fill_shared_expert_slot(P, P, 4, 9, 256, 1, None, 2.5, None) == 1    # no picks
+    assert lib.moe_fill_shared_expert_slot(P, P, 4, 9, 256, 1, P, float("nan"), None) == 1
+    assert lib.moe_fill_shared_expert_slot(P, P, 0, 9, 256, 1, None, 2.5, None) == 0    # empty: no launch
+    assert lib.moe_sort_topk_by_id(P, None, 4, 8, None) == 1
+    assert lib.moe_sort_topk_by_id(P, P, 4, 40, None) == 2
+    assert lib.moe_sort_topk_by_id(P, P, 0, 8, None) == 0

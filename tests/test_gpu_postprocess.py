@@ -1,0 +1,67 @@
+"""Shared-expert slot fill and ascending-id order on routing results, against
+the oracle, through the C ABI (GPU only)."""
+import numpy as np
+import pytest
+import torch
+
+import moe_expert_routing_token_b200 as moe
+import oracle
+from moe_expert_routing_token_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _routed(M, k, seed):
+    """A DeepSeek-V3 style result: 8 routed experts + one slot for the shared expert."""
+    d = inputs.make("biased", M, seed=seed)
+    w, ids = moe.biased_grouped_topk(d["logits"].to(DEV), d["bias"].to(DEV), k, True, 8, 4, 2.5)
+    return w, ids
+
+
+@pytest.mark.parametrize("M,k", [(1, 9), (1000, 9), (16384, 9), (333, 1), (257, 32)])
+@pytest.mark.parametrize("rsf", [2.5, None])
+def test_fill_shared_expert_slot(M, k, rsf):
+    if k == 32:
+        g = torch.Generator().manual_seed(M)
+        w = torch.rand(M, k, generator=g).to(DEV)
+        ids = torch.randint(0, 256, (M, k), generator=g, dtype=torch.int32).to(DEV)
+    else:
+        w, ids = _routed(M, k, seed=M + k)
+    num_shared = 3
+    pick = torch.randint(0, num_shared, (M,), generator=torch.Generator().manual_seed(7),
+                         dtype=torch.int32).to(DEV)
+    w0, ids0 = w.cpu().numpy(), ids.cpu().numpy()
+    moe.fill_shared_expert_slot(w, ids, 256, num_shared, pick, rsf)
+    torch.cuda.synchronize()
+    w_ref, ids_ref = oracle.fill_shared_slot(w0, ids0, 256, num_shared, pick.cpu().numpy(), rsf)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    got = w.cpu().numpy().astype(np.float64)
+    assert np.array_equal(got[:, :-1], w0[:, :-1].astype(np.float64))       # other slots untouched
+    assert np.allclose(got[:, -1], w_ref[:, -1], rtol=1e-6, atol=0.0)
+
+
+@pytest.mark.parametrize("M,k", [(1, 8), (5000, 8), (16384, 9), (700, 1), (129, 32)])
+def test_sort_topk_by_id(M, k):
+    g = torch.Generator().manual_seed(M * 3 + k)
+    if k in (8, 9):
+        w, ids = _routed(M, k, seed=M)
+    else:
+        w = torch.rand(M, k, generator=g).to(DEV)
+        ids = torch.randint(0, 16, (M, k), generator=g, dtype=torch.int32).to(DEV)   # repeated ids
+    w0, ids0 = w.cpu().numpy(), ids.cpu().numpy()
+    moe.sort_topk_by_id(w, ids)
+    torch.cuda.synchronize()
+    w_ref, ids_ref = oracle.sort_by_id(w0, ids0)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    assert np.array_equal(w.cpu().numpy().astype(np.float64), w_ref)       # a permutation: exact
+
+
+def test_fill_then_sort_composes():
+    w, ids = _routed(4096, 9, seed=5)
+    pick = torch.zeros(4096, dtype=torch.int32, device=DEV)
+    moe.fill_shared_expert_slot(w, ids, 256, 1, pick, 2.5)
+    moe.sort_topk_by_id(w, ids)
+    torch.cuda.synchronize()
+    ids_h = ids.cpu().numpy()
+    assert np.all(np.diff(ids_h, axis=1) >= 0) and np.all(ids_h[:, -1] == 256)
