@@ -143,8 +143,8 @@ MOE_API int moe_grouped_topk(const void* gating_output, int dtype, int64_t M, in
  * the plain sigmoid(+bias) top-k of sgl_kernel topk_sigmoid.
  *
  *   correction_bias  device, (E,) fp32, or NULL for no bias.  It stays fp32
- *                    (the aiter path casts it to the logits dtype; this
- *                    library does not).
+ *                    (the aiter path casts it to the logits dtype: see
+ *                    moe_biased_grouped_topk_aiter).
  *   other arguments as moe_grouped_topk
  */
 MOE_API int moe_biased_grouped_topk(const void* gating_output, int dtype,
@@ -153,6 +153,19 @@ MOE_API int moe_biased_grouped_topk(const void* gating_output, int dtype,
                             int32_t num_expert_group, int32_t topk_group,
                             float routed_scaling_factor, float* topk_weights,
                             int32_t* topk_ids, void* stream);
+
+/*
+ * moe_biased_grouped_topk_aiter - moe_biased_grouped_topk with the aiter
+ * path's bias handling ([A] 코드 분석, After: aiter_biased_grouped_topk is
+ * handed correction_bias.to(gating_output.dtype)): with bf16 logits the bias
+ * is rounded to bf16 (round to nearest even) before it is added; with fp32
+ * logits the two calls are identical.  Arguments as moe_biased_grouped_topk.
+ */
+MOE_API int moe_biased_grouped_topk_aiter(const void* gating_output, int dtype, const float* correction_bias,
+                                          int64_t M, int32_t E, int32_t topk, int32_t renormalize,
+                                          int32_t num_expert_group, int32_t topk_group,
+                                          float routed_scaling_factor, float* topk_weights, int32_t* topk_ids,
+                                          void* stream);
 
 /*
  * moe_fused_router_workspace_size - bytes of device workspace that

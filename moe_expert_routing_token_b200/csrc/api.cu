@@ -254,7 +254,7 @@ int dispatch_typed(const RouteArgs& a, cudaStream_t st) {
 
 int route(const void* logits, int dtype, const float* bias, int64_t M, int E, int K, int renorm,
           int G, int TG, int group_kind, int scoring, float rsf, float* weights, int32_t* ids,
-          void* stream, const char* who) {
+          void* stream, const char* who, int bias_bf16 = 0) {
     if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16)
         return fail(MOE_ERR_INVALID_ARG, "%s: dtype %d is neither MOE_DTYPE_F32 nor MOE_DTYPE_BF16", who, dtype);
     if (M < 0) return fail(MOE_ERR_INVALID_ARG, "%s: M=%lld < 0", who, (long long)M);
@@ -287,6 +287,7 @@ int route(const void* logits, int dtype, const float* bias, int64_t M, int E, in
     a.rsf = rsf;
     a.weights = weights;
     a.ids = ids;
+    a.bias_bf16 = (bias_bf16 && dtype == MOE_DTYPE_BF16) ? 1 : 0;  // an fp32 cast of fp32 logits changes nothing
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     if (scoring == kSoftmax) {
@@ -373,6 +374,17 @@ int moe_biased_grouped_topk(const void* gating_output, int dtype, const float* c
                       num_expert_group, topk_group, moe::kGroupTop2Sum, moe::kSigmoid,
                       routed_scaling_factor, topk_weights, topk_ids, stream,
                       "moe_biased_grouped_topk");
+}
+
+int moe_biased_grouped_topk_aiter(const void* gating_output, int dtype, const float* correction_bias,
+                                  int64_t M, int32_t E, int32_t topk, int32_t renormalize,
+                                  int32_t num_expert_group, int32_t topk_group,
+                                  float routed_scaling_factor, float* topk_weights, int32_t* topk_ids,
+                                  void* stream) {
+    return moe::route(gating_output, dtype, correction_bias, M, E, topk, renormalize,
+                      num_expert_group, topk_group, moe::kGroupTop2Sum, moe::kSigmoid,
+                      routed_scaling_factor, topk_weights, topk_ids, stream,
+                      "moe_biased_grouped_topk_aiter", 1);
 }
 
 }  // extern "C"

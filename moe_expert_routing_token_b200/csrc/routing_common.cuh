@@ -30,7 +30,14 @@ struct RouteArgs {
     float rsf;            // routed_scaling_factor
     float* weights;       // (M, K) fp32
     int32_t* ids;         // (M, K) int32
+    int bias_bf16 = 0;    // 1: round the bias to bf16 before use (the aiter variant)
 };
+
+// The correction bias as the kernels use it: fp32, or (aiter variant, bf16
+// logits) rounded to the logits dtype first.
+__device__ __forceinline__ float bias_as_used(float b, int round_bf16) {
+    return round_bf16 ? __bfloat162float(__float2bfloat16_rn(b)) : b;
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

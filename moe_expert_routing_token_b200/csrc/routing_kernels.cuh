@@ -80,8 +80,9 @@ struct SegRouter {
 
     // Copy the (E,) bias from global memory into the padded layout; called
     // by every thread of the block, followed by a barrier.
-    __device__ __forceinline__ static void load_bias_padded(const float* g_bias, float* s_bias) {
-        for (int e = threadIdx.x; e < E; e += blockDim.x) s_bias[(e / C) * CS + e % C] = __ldg(g_bias + e);
+    __device__ __forceinline__ static void load_bias_padded(const float* g_bias, float* s_bias, int round_bf16) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x)
+            s_bias[(e / C) * CS + e % C] = bias_as_used(__ldg(g_bias + e), round_bf16);
     }
 
     // Unbiased scores kept in a per-warp shared buffer (for callers whose raw
@@ -353,7 +354,7 @@ __global__ void __launch_bounds__(kSegThreads) route_segment_kernel(RouteArgs a)
     ptx::griddep_launch_dependents();
     ptx::griddep_wait();
     if constexpr (BIAS) {
-        Router::load_bias_padded(a.bias, s_bias);
+        Router::load_bias_padded(a.bias, s_bias, a.bias_bf16);
         __syncthreads();
     }
 
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs a) {
 #pragma unroll
         for (int i = 0; i < E; ++i) {
             p[i] = (SCORE == kSigmoid) ? sigmoid_f32(x[i]) : x[i];
-            key[i] = BIAS ? p[i] + __ldg(a.bias + i) : p[i];
+            key[i] = BIAS ? p[i] + bias_as_used(__ldg(a.bias + i), a.bias_bf16) : p[i];
             mx = fmaxf(mx, x[i]);
         }
         // admissible experts: those of the TG best groups
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(128) route_generic_kernel(RouteArgs a) {
             const float x = load_scalar<TIn>(logits + row * E + e);
             const float p = (SCORE == kSigmoid) ? sigmoid_f32(x) : x;
             s_p[e] = p;
-            s_key[e] = (a.bias != nullptr) ? p + __ldg(a.bias + e) : p;
+            s_key[e] = (a.bias != nullptr) ? p + bias_as_used(__ldg(a.bias + e), a.bias_bf16) : p;
             mx = fmaxf(mx, x);
         }
 #pragma unroll

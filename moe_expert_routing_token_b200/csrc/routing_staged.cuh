@@ -107,7 +107,7 @@ __global__ void __launch_bounds__((kStagedWarps + 1) * 32)
     // Everything above overlaps the previous kernel in the stream; global
     // inputs are read only after it has finished.
     ptx::griddep_wait();
-    if constexpr (BIAS) Router::load_bias_padded(a.bias, s_bias);
+    if constexpr (BIAS) Router::load_bias_padded(a.bias, s_bias, a.bias_bf16);
     __syncthreads();
 
     if (warp == W) {

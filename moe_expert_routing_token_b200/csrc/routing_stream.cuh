@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     auto build_tables = [&]() {
         float bmax = 0.0f;
         for (int e = lane; e < E; e += 32) {
-            const float b = BIAS ? __ldg(a.bias + e) : 0.0f;
+            const float b = BIAS ? bias_as_used(__ldg(a.bias + e), a.bias_bf16) : 0.0f;
             s_b2[e] = b;
             s_b1[(e / C) * CS + e % C] = APPROX ? 0.5f + b : b;
             bmax = fmaxf(bmax, fabsf(b));

@@ -41,6 +41,8 @@ SIGNATURES = {
                                         _vp, _vp, _vp]),
     "moe_biased_grouped_topk": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32, _i32,
                                                _i32, _f32, _vp, _vp, _vp]),
+    "moe_biased_grouped_topk_aiter": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32, _i32,
+                                               _i32, _f32, _vp, _vp, _vp]),
     "moe_fused_router_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_fused_router_topk": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32, _i32,
                                              _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -156,17 +158,20 @@ def grouped_topk(gating_output: torch.Tensor, topk: int, renormalize: bool, num_
 
 def biased_grouped_topk(gating_output: torch.Tensor, correction_bias, topk: int,
                         renormalize: bool, num_expert_group: int = 1, topk_group: int = 1,
-                        routed_scaling_factor: float = 1.0, out=None):
+                        routed_scaling_factor: float = 1.0, out=None, bias_as_logits_dtype: bool = False):
     """Sigmoid + correction_bias grouped top-k (group score = sum of top-2).
-    With num_expert_group = topk_group = 1 it is the sigmoid top-k."""
+    With num_expert_group = topk_group = 1 it is the sigmoid top-k.
+    bias_as_logits_dtype: the aiter variant (moe_biased_grouped_topk_aiter),
+    the bias rounded to bf16 logits' dtype before it is added."""
     _cuda_2d(gating_output, "gating_output")
     M, E = gating_output.shape
     bp = _bias_ptr(correction_bias, E, gating_output.device)
     w, ids = _outputs(M, topk, gating_output.device, out)
-    st = lib().moe_biased_grouped_topk(gating_output.data_ptr(), _dtype_code(gating_output), bp, M, E,
-                                       topk, int(bool(renormalize)), num_expert_group, topk_group,
-                                       float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
-                                       _stream(gating_output.device))
+    fn = lib().moe_biased_grouped_topk_aiter if bias_as_logits_dtype else lib().moe_biased_grouped_topk
+    st = fn(gating_output.data_ptr(), _dtype_code(gating_output), bp, M, E,
+            topk, int(bool(renormalize)), num_expert_group, topk_group,
+            float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
+            _stream(gating_output.device))
     _check(st, "moe_biased_grouped_topk")
     return w, ids
 

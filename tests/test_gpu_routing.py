@@ -209,3 +209,39 @@ def test_no_watchdog_trips():
     """No kernel gave up on a barrier wait during the tests above."""
     torch.cuda.synchronize()
     assert moe.watchdog_trips() == 0
+
+
+@pytest.mark.parametrize("M,E,G,TG,k", [(2048, 256, 1, 1, 8),    # streaming kernel (approximate keys)
+                                        (2048, 256, 8, 4, 8),    # streaming kernel (exact keys)
+                                        (2048, 256, 8, 8, 16),   # staged kernel (k > 8)
+                                        (500, 256, 8, 4, 8),     # segment kernel
+                                        (600, 32, 4, 2, 5),      # small-E kernel
+                                        (700, 128, 16, 4, 8)])   # generic kernel
+def test_aiter_bias_cast_variant(M, E, G, TG, k):
+    """moe_biased_grouped_topk_aiter rounds the fp32 bias to the bf16 logits'
+    dtype first: it must match the oracle on the rounded bias, and biases in
+    [0.25, 0.5] (rounding error up to ~5e-4, above the key gaps near the top)
+    make it differ from the fp32-bias call on clear rows."""
+    g = torch.Generator().manual_seed(E * 13 + k)
+    x = (torch.randn(M, E, generator=g) * 0.5).to(torch.bfloat16)
+    bias = 0.25 + 0.25 * torch.rand(E, generator=g)
+    xd, bd = x.to(DEV), bias.to(DEV)
+    w, ids = moe.biased_grouped_topk(xd, bd, k, True, G, TG, 2.5, bias_as_logits_dtype=True)
+    w2, ids2 = moe.biased_grouped_topk(xd, bd, k, True, G, TG, 2.5)
+    torch.cuda.synchronize()
+    b16 = bias.to(torch.bfloat16).to(torch.float32)
+    orc = run_oracle("sigmoid", x, b16, k, True, G, TG, 2.5)
+    rep = parity.compare(w.cpu().numpy(), ids.cpu().numpy(), orc, E=E, G=G, TG=TG, k=k, renorm=True, rsf=2.5,
+                         fp32_logits=False)
+    assert rep.ok(), rep.summary()
+    assert not torch.equal(ids, ids2), "rounding the bias changed no routing decision"
+
+
+def test_aiter_variant_is_the_plain_call_for_fp32_logits():
+    d = inputs.make("grouped", 3000)
+    x = d["logits"].to(DEV)
+    bias = inputs.random_bias(160, 0.05, seed=3).to(DEV)
+    a = moe.biased_grouped_topk(x, bias, 6, True, 8, 3, 1.0, bias_as_logits_dtype=True)
+    b = moe.biased_grouped_topk(x, bias, 6, True, 8, 3, 1.0)
+    torch.cuda.synchronize()
+    assert torch.equal(a[1], b[1]) and torch.equal(a[0], b[0])
