@@ -7,20 +7,22 @@
 // gathered weights being the unbiased scores, renormalised and scaled.  Ties
 // go to the lower expert / group index and ids leave in descending score.
 //
-// Three kernels, picked by shape:
+// This file holds the SegRouter routing body and three kernels (the
+// streaming kernels for large batches are in routing_stream.cuh, k <= 8, and
+// routing_staged.cuh, k > 8):
 //
-//  * route_segment_kernel (the hot path, E = 160 or 256): a row is owned by a
-//    segment of L = E / C lanes, each lane holding C consecutive experts in
-//    registers after one pass of 16-byte loads.  A lane's chunk never
-//    straddles a group, so group scores need only xor-shuffles among the
-//    group's lanes.  Instead of k rounds of arg-max, the kernel derives a
-//    threshold tau that the k-th best admissible score is known to reach (the
-//    ceil(k/2)-th best per-lane second-largest score among kept lanes: those
-//    lanes alone hold k admissible experts >= tau), collects the few
-//    candidates >= tau into shared memory, and ranks each candidate by
-//    counting how many candidates beat it - the ballot/popcount rank idea of
-//    the MiniMax-M3 page's warp rank sort, applied to scores.  Rows with more
-//    than kCandCap candidates (massive ties) take an exact k-round arg-max.
+//  * route_segment_kernel (E = 160 or 256, batches below 1024 rows): a row is
+//    owned by a segment of L = E / C lanes, each lane holding C consecutive
+//    experts in registers after one pass of 16-byte loads.  A lane's chunk
+//    never straddles a group, so group scores need only xor-shuffles among
+//    the group's lanes.  Instead of k rounds of arg-max, the kernel derives a
+//    threshold tau that the k-th best admissible score is known to reach (for
+//    k <= 8 the k-th largest of the kept lanes' top-2 values: they are k
+//    distinct admissible experts), collects the few candidates >= tau into
+//    shared memory, and ranks each candidate by counting how many candidates
+//    beat it - the ballot/popcount rank idea of the MiniMax-M3 page's warp
+//    rank sort, applied to scores.  Rows with more than kCandCap candidates
+//    (massive ties) take an exact k-round arg-max.
 //  * route_small_kernel (E <= 32): one thread per row, k rounds of arg-max in
 //    registers.
 //  * route_generic_kernel (any E <= 1024, any group shape, any alignment): one
