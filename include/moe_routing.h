@@ -134,6 +134,21 @@ MOE_API int moe_grouped_topk(const void* gating_output, int dtype, int64_t M, in
                      float* topk_weights, int32_t* topk_ids, void* stream);
 
 /*
+ * moe_grouped_topk_softcap - moe_grouped_topk with the logit softcapping of
+ * the fused router ([R] §5: logits / c -> tanh -> * c when moe_softcapping is
+ * nonzero).  c * tanh(x / c) is strictly increasing, so the experts chosen
+ * are those of moe_grouped_topk; the weights are the softmax of the capped
+ * logits (renormalised over the k or over all experts, then scaled).  With
+ * topk = 1 and renormalize = 0 the weight is the top-1 probability
+ * 1 / sum(exp(capped - capped max)) of the same section.  softcap 0 = none;
+ * it must be finite.  Other arguments as moe_grouped_topk.
+ */
+MOE_API int moe_grouped_topk_softcap(const void* gating_output, int dtype, int64_t M, int32_t E, int32_t topk,
+                                     int32_t renormalize, int32_t num_expert_group, int32_t topk_group,
+                                     float routed_scaling_factor, float softcap, float* topk_weights,
+                                     int32_t* topk_ids, void* stream);
+
+/*
  * moe_biased_grouped_topk - [R] §4 (DeepSeek-V3 biased_grouped_topk_impl) and
  * [A] (aiter biased_grouped_topk): sigmoid scores; selection score = score +
  * correction_bias; group score = sum of the group's two largest selection

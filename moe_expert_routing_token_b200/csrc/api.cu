@@ -254,7 +254,7 @@ int dispatch_typed(const RouteArgs& a, cudaStream_t st) {
 
 int route(const void* logits, int dtype, const float* bias, int64_t M, int E, int K, int renorm,
           int G, int TG, int group_kind, int scoring, float rsf, float* weights, int32_t* ids,
-          void* stream, const char* who, int bias_bf16 = 0) {
+          void* stream, const char* who, int bias_bf16 = 0, float softcap = 0.0f) {
     if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16)
         return fail(MOE_ERR_INVALID_ARG, "%s: dtype %d is neither MOE_DTYPE_F32 nor MOE_DTYPE_BF16", who, dtype);
     if (M < 0) return fail(MOE_ERR_INVALID_ARG, "%s: M=%lld < 0", who, (long long)M);
@@ -288,6 +288,8 @@ int route(const void* logits, int dtype, const float* bias, int64_t M, int E, in
     a.weights = weights;
     a.ids = ids;
     a.bias_bf16 = (bias_bf16 && dtype == MOE_DTYPE_BF16) ? 1 : 0;  // an fp32 cast of fp32 logits changes nothing
+    if (!std::isfinite(softcap)) return fail(MOE_ERR_INVALID_ARG, "%s: softcap is not finite", who);
+    a.softcap = (scoring == kSoftmax) ? softcap : 0.0f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     if (scoring == kSoftmax) {
@@ -374,6 +376,15 @@ int moe_biased_grouped_topk(const void* gating_output, int dtype, const float* c
                       num_expert_group, topk_group, moe::kGroupTop2Sum, moe::kSigmoid,
                       routed_scaling_factor, topk_weights, topk_ids, stream,
                       "moe_biased_grouped_topk");
+}
+
+int moe_grouped_topk_softcap(const void* gating_output, int dtype, int64_t M, int32_t E, int32_t topk,
+                             int32_t renormalize, int32_t num_expert_group, int32_t topk_group,
+                             float routed_scaling_factor, float softcap, float* topk_weights, int32_t* topk_ids,
+                             void* stream) {
+    return moe::route(gating_output, dtype, nullptr, M, E, topk, renormalize, num_expert_group, topk_group,
+                      moe::kGroupMax, moe::kSoftmax, routed_scaling_factor, topk_weights, topk_ids, stream,
+                      "moe_grouped_topk_softcap", 0, softcap);
 }
 
 int moe_biased_grouped_topk_aiter(const void* gating_output, int dtype, const float* correction_bias,

@@ -31,7 +31,10 @@ struct RouteArgs {
     float* weights;       // (M, K) fp32
     int32_t* ids;         // (M, K) int32
     int bias_bf16 = 0;    // 1: round the bias to bf16 before use (the aiter variant)
+    float softcap = 0.0f; // softmax: weights from c * tanh(x / c) (0: none)
 };
+
+
 
 // The correction bias as the kernels use it: fp32, or (aiter variant, bf16
 // logits) rounded to the logits dtype first.
@@ -103,6 +106,17 @@ __device__ __forceinline__ float exp_f32(float x) {
     float e;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * 1.4426950408889634f));
     return e;
+}
+
+// Logit softcapping of the fused router (routing page §5): c * tanh(x / c),
+// with the accurate tanhf; c = 0 leaves x as it is.  It is strictly
+// increasing, so selection on the raw logits picks the same experts; only the
+// softmax weights and denominators use the capped values.
+__device__ __forceinline__ float softcap_f32(float x, float c) { return c != 0.0f ? c * tanhf(x / c) : x; }
+
+// exp(cap(v) - cap(vmax)), the softmax numerator relative to the row max.
+__device__ __forceinline__ float softmax_num(float v, float vmax, float c) {
+    return exp_f32(softcap_f32(v, c) - softcap_f32(vmax, c));
 }
 
 // Three-input max / min (sm_100).

@@ -293,7 +293,7 @@ struct SegRouter {
             if (!a.renorm) {
                 float s = 0.0f;
 #pragma unroll
-                for (int i = 0; i < C; ++i) s += exp_f32(key[i] - rowmax);
+                for (int i = 0; i < C; ++i) s += softmax_num(key[i], rowmax, a.softcap);
 #pragma unroll
                 for (int o = L / 2; o >= 1; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
                 denom_all = s;
@@ -309,7 +309,7 @@ struct SegRouter {
             id_loc[q] = 0;
             if (t < K) {
                 const float2 o = sc.out[seg][t];
-                const float w = (SCORE == kSoftmax) ? exp_f32(o.x - rowmax) : o.x;
+                const float w = (SCORE == kSoftmax) ? softmax_num(o.x, rowmax, a.softcap) : o.x;
                 w_loc[q] = w;
                 id_loc[q] = __float_as_int(o.y);
                 sum += w;
@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs a) {
         if (SCORE == kSoftmax && !a.renorm) {
             float s = 0.0f;
 #pragma unroll
-            for (int i = 0; i < E; ++i) s += exp_f32(x[i] - mx);
+            for (int i = 0; i < E; ++i) s += softmax_num(x[i], mx, a.softcap);
             denom_all = s;
         }
         float sum = 0.0f;
@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(RouteArgs a) {
             }
             if (bi < 0) bi = 0;  // unreachable for valid arguments
             taken |= 1u << bi;
-            const float w = (SCORE == kSoftmax) ? exp_f32(bp - mx) : bp;
+            const float w = (SCORE == kSoftmax) ? softmax_num(bp, mx, a.softcap) : bp;
             sum += w;
             a.weights[row * K + j] = w;
             a.ids[row * K + j] = bi;
@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(128) route_generic_kernel(RouteArgs a) {
         float denom_all = 1.0f;
         if (SCORE == kSoftmax && !a.renorm) {
             float s = 0.0f;
-            for (int e = lane; e < E; e += 32) s += exp_f32(s_p[e] - mx);
+            for (int e = lane; e < E; e += 32) s += softmax_num(s_p[e], mx, a.softcap);
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
             denom_all = s;
@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(128) route_generic_kernel(RouteArgs a) {
                 }
             }
             if (bi == 0x7fffffff) bi = 0;  // unreachable for valid arguments
-            const float w = (SCORE == kSoftmax) ? exp_f32(s_p[bi] - mx) : s_p[bi];
+            const float w = (SCORE == kSoftmax) ? softmax_num(s_p[bi], mx, a.softcap) : s_p[bi];
             sum += w;
             if (lane == j) {
                 my_w = w;

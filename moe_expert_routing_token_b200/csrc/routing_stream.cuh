@@ -232,7 +232,7 @@ __device__ __forceinline__ void route_stream_phase2(const RouteArgs& a, int64_t 
         for (int q = 0; q < 8; ++q) {
             wv[q] = 0.0f;
             if (q < K) {
-                wv[q] = (SCORE == kSoftmax) ? exp_f32(xw[q] - rowmax) : sigmoid_f32(xw[q]);
+                wv[q] = (SCORE == kSoftmax) ? softmax_num(xw[q], rowmax, a.softcap) : sigmoid_f32(xw[q]);
                 sum += wv[q];
             }
         }
@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 if (!a.renorm) {
                     float sacc = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < C; ++i) sacc += exp_f32(x[i] - mx);
+                    for (int i = 0; i < C; ++i) sacc += softmax_num(x[i], mx, a.softcap);
 #pragma unroll
                     for (int o = L / 2; o >= 1; o >>= 1) sacc += __shfl_xor_sync(kFullMask, sacc, o);
                     den = sacc;

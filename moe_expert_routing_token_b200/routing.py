@@ -43,6 +43,8 @@ SIGNATURES = {
                                                _i32, _f32, _vp, _vp, _vp]),
     "moe_biased_grouped_topk_aiter": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32, _i32,
                                                _i32, _f32, _vp, _vp, _vp]),
+    "moe_grouped_topk_softcap": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _i32, _i32, _i32, _i32, _f32,
+                                                _f32, _vp, _vp, _vp]),
     "moe_fused_router_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_fused_router_topk": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32, _i32,
                                              _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -143,11 +145,20 @@ def topk_softmax(gating_output: torch.Tensor, topk: int, renormalize: bool, out=
 
 
 def grouped_topk(gating_output: torch.Tensor, topk: int, renormalize: bool, num_expert_group: int,
-                 topk_group: int, routed_scaling_factor: float = 1.0, out=None):
-    """Softmax grouped top-k (group score = max).  Returns (weights, ids)."""
+                 topk_group: int, routed_scaling_factor: float = 1.0, out=None, softcap: float = 0.0):
+    """Softmax grouped top-k (group score = max).  Returns (weights, ids).
+    softcap != 0: weights from the softmax of softcap * tanh(logits / softcap)
+    (moe_grouped_topk_softcap)."""
     _cuda_2d(gating_output, "gating_output")
     M, E = gating_output.shape
     w, ids = _outputs(M, topk, gating_output.device, out)
+    if softcap:
+        st = lib().moe_grouped_topk_softcap(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
+                                            int(bool(renormalize)), num_expert_group, topk_group,
+                                            float(routed_scaling_factor), float(softcap), w.data_ptr(),
+                                            ids.data_ptr(), _stream(gating_output.device))
+        _check(st, "moe_grouped_topk_softcap")
+        return w, ids
     st = lib().moe_grouped_topk(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
                                 int(bool(renormalize)), num_expert_group, topk_group,
                                 float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),

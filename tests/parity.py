@@ -53,7 +53,7 @@ class Report:
 
 
 def compare(w_gpu, ids_gpu, orc, *, E: int, G: int, TG: int, k: int, renorm: bool, rsf: float,
-            fp32_logits: bool, rows=None, eps: float = EPS) -> Report:
+            fp32_logits: bool, rows=None, eps: float = EPS, w_rtol: float | None = None) -> Report:
     """Compare GPU outputs (numpy or CPU tensors) with an oracle Routing.
 
     ``rows``: optional index array - the GPU rows that the oracle rows
@@ -130,7 +130,9 @@ def compare(w_gpu, ids_gpu, orc, *, E: int, G: int, TG: int, k: int, renorm: boo
     expect = pw * rsf
     err = np.abs(w_gpu - expect)
     rep.max_weight_err = float(err.max())
-    if fp32_logits:
+    if w_rtol is not None:  # a tolerance the caller derives for its arithmetic
+        bad = err > w_rtol * np.abs(expect) + 1e-30
+    elif fp32_logits:
         bad = err > ABS_TOL_F32
     else:
         bad = err > REL_TOL_BF16 * np.abs(expect) + 1e-30

@@ -245,3 +245,37 @@ def test_aiter_variant_is_the_plain_call_for_fp32_logits():
     b = moe.biased_grouped_topk(x, bias, 6, True, 8, 3, 1.0)
     torch.cuda.synchronize()
     assert torch.equal(a[1], b[1]) and torch.equal(a[0], b[0])
+
+
+@pytest.mark.parametrize("M,E,G,TG,k,renorm", [(2048, 256, 1, 1, 8, True),    # streaming kernel
+                                               (2048, 160, 8, 3, 6, False),   # streaming, full denominators
+                                               (2048, 256, 8, 8, 16, True),   # staged kernel (k > 8)
+                                               (500, 256, 8, 4, 8, False),    # segment kernel
+                                               (600, 8, 1, 1, 1, False),      # small-E: top-1 = 1 / sum exp
+                                               (700, 64, 8, 3, 5, True)])     # generic kernel
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_softcapped_softmax(M, E, G, TG, k, renorm, dtype):
+    """moe_grouped_topk_softcap: the oracle's softmax routing of the capped
+    logits 30 * tanh(x / 30) (computed in double).  Weight tolerance for fp32
+    logits: tanhf's ~2 ulp, times c, plus roundings, gives ~4e-7 * c on each
+    capped logit and, through exp and the sum, below 1.4e-5 relative; 2e-5."""
+    c = 30.0
+    x = inputs.random_logits(M, E, 20.0, dtype, seed=E + k + M)
+    w, ids = moe.grouped_topk(x.to(DEV), k, renorm, G, TG, 1.5, softcap=c)
+    torch.cuda.synchronize()
+    xc = c * np.tanh(oracle.as_f64(x) / c)
+    orc = oracle.grouped_topk(xc, k, renorm, G, TG, 1.5)
+    rep = parity.compare(w.cpu().numpy(), ids.cpu().numpy(), orc, E=E, G=G, TG=TG, k=k, renorm=renorm, rsf=1.5,
+                         fp32_logits=(dtype == torch.float32),
+                         w_rtol=2e-5 if dtype == torch.float32 else None)
+    assert rep.ok(), rep.summary()
+
+
+def test_softcap_zero_is_the_plain_call():
+    x = inputs.random_logits(3000, 256, 3.0, torch.bfloat16, seed=8).to(DEV)
+    a = moe.grouped_topk(x, 8, True, 8, 4, 1.0)
+    b = torch.empty_like(a[0]), torch.empty_like(a[1])
+    st = moe.lib().moe_grouped_topk_softcap(x.data_ptr(), 1, 3000, 256, 8, 1, 8, 4, 1.0, 0.0, b[0].data_ptr(),
+                                            b[1].data_ptr(), torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert st == 0 and torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
