@@ -66,7 +66,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1, /* argument outside the documented domain     */
-    MOE_ERR_UNSUPPORTED = 2, /* valid, but this build has no kernel for it */
+    MOE_ERR_UNSUPPORTED = 2, /* valid, but the library has no kernel for it */
     MOE_ERR_CUDA = 3         /* the CUDA runtime reported an error         */
 } moe_status_t;
 
@@ -203,7 +203,7 @@ MOE_API size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E);
  *                   or (E, K) if MOE_WEIGHT_E_BY_K
  *   correction_bias device, (E,) fp32, or NULL
  *   K               hidden size, a positive multiple of 64
- *   E               experts; this build supports E == 256
+ *   E               experts; the fused router is built for E == 256
  *   logits_out      device, (M, E) fp32 out, or NULL (debug: the fp32 logits
  *                   the routing consumed)
  *   workspace       device scratch of at least

@@ -664,7 +664,7 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
         return set_error(MOE_ERR_INVALID_ARG, msg);
     }
     if (E != 256) {
-        snprintf(msg, sizeof msg, "%s: E=%d; this build supports E=256", who, E);
+        snprintf(msg, sizeof msg, "%s: E=%d; the fused router is built for E=256", who, E);
         return set_error(MOE_ERR_UNSUPPORTED, msg);
     }
     if (K % 64 != 0) {
