@@ -1,0 +1,28 @@
+"""bench.py's reference arm (the oracle on the host cores) prints the one-line
+JSON record the benchmark contract asks for (CPU only)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+        "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
+
+
+@pytest.mark.parametrize("workload", ["sigmoid", "permute"])
+def test_reference_arm_record(workload):
+    res = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", workload,
+                          "--steps", "2", "--warmup", "1", "--cpu-seconds", "0.5"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert KEYS <= set(rec), KEYS - set(rec)
+    assert rec["impl"] == "reference" and rec["value"] > 0 and rec["higher_is_better"] is True
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] == 1
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
+    assert isinstance(rec["config"], dict) and "workload" in rec["config"]
