@@ -320,6 +320,17 @@ MOE_API int moe_fill_shared_expert_slot(float* topk_weights, int32_t* topk_ids, 
  */
 MOE_API int moe_sort_topk_by_id(float* topk_weights, int32_t* topk_ids, int64_t M, int32_t k, void* stream);
 
+/*
+ * moe_selftest_bounded_wait - checks the failure path of the library's
+ * bounded waits without a fault: one thread waits on an mbarrier that nothing
+ * completes, with a budget of budget_ns (0 < budget_ns <= 1e9), gives up and
+ * writes status[0] = 1 (0 if the wait had completed) and status[1] = the
+ * microseconds it waited.  status: device int32[2].  The routing kernels use
+ * the same wait (with a 2 s budget) and count a give-up in
+ * moe_watchdog_trips; this call touches no counter.
+ */
+MOE_API int moe_selftest_bounded_wait(uint64_t budget_ns, int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -53,6 +53,7 @@ SIGNATURES = {
     "moe_expert_permutation_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_fill_shared_expert_slot": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _i32, _vp, _f32, _vp]),
     "moe_sort_topk_by_id": (ctypes.c_int, [_vp, _vp, _i64, _i32, _vp]),
+    "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, _vp, _vp]),
     "moe_expert_permutation": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                               _vp]),
 }
