@@ -55,7 +55,11 @@
 extern "C" {
 #endif
 
-#define MOE_ROUTING_ABI_VERSION 1
+/* 1: the routing calls and the fused router.  2: adds the allocation-free
+ * fused router, the softcap and aiter variants, the expert permutation, the
+ * shared-expert slot, the ascending-id order and the bounded-wait self-test
+ * (every version-1 call keeps its signature and meaning). */
+#define MOE_ROUTING_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
     assert lib.moe_status_string(0) == b"MOE_OK"
     assert lib.moe_status_string(1) == b"MOE_ERR_INVALID_ARG"
     assert lib.moe_status_string(2) == b"MOE_ERR_UNSUPPORTED"
