@@ -44,7 +44,6 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kEpiWarps = 16;                // four per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kFinStride = 8 * 36 + 4;  // floats per staged row: 8 chunks of 36 (bank spread)
-constexpr int kPrefetchAhead = 6;       // k-blocks of A brought into L2 ahead of their load
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 using Router = SegRouter<256, 32, kSigmoid, true>;
@@ -202,12 +201,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t* a_s = smem + (size_t)s * kStageBytes;
                 uint8_t* b_s = a_s + kABytes;
                 const int kc = (kb0 + kb) * kBK;
-                if (kb == 0) {
-                    for (int j = 1; j <= kPrefetchAhead && j < nkb; ++j)
-                        ptx::tma_prefetch_l2_2d(&tmA, (kb0 + j) * kBK, m_tile * kBM);
-                } else if (kb + kPrefetchAhead < nkb) {
-                    ptx::tma_prefetch_l2_2d(&tmA, (kb0 + kb + kPrefetchAhead) * kBK, m_tile * kBM);
-                }
                 ptx::mbar_arrive_expect_tx(&full[s], kStageBytes);
                 ptx::tma_load_2d(a_s, &tmA, kc, m_tile * kBM, &full[s], pol_a);
                 if constexpr (B_MN_MAJOR) {
