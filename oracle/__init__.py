@@ -19,6 +19,9 @@ Operations (each a restatement of the SGLang MoE routing page,
 * :func:`router_logits`       - §5 router projection, exact products summed
   in double
 * :func:`fused_router_topk`   - §5 projection followed by §4 routing
+* :func:`softcap_logits`      - §5 softcapping, c * tanh(logits / c)
+* :func:`fused_router_top1`   - §5 projection, softcapping and softmax top-1
+  (weight = 1 / sum_e exp(l_e - max l), the page's invsumexp)
 """
 from __future__ import annotations
 
@@ -64,6 +67,8 @@ def _bind(path: str):
     lib.oracle_router_logits.restype = ctypes.c_int
     lib.oracle_router_logits.argtypes = [
         _DBL, _DBL, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _DBL]
+    lib.oracle_softcap.restype = ctypes.c_int
+    lib.oracle_softcap.argtypes = [_DBL, ctypes.c_int64, ctypes.c_double, _DBL]
     lib.oracle_fill_shared_slot.restype = ctypes.c_int
     lib.oracle_fill_shared_slot.argtypes = [_DBL, _I32, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             _I32, ctypes.c_double]
@@ -191,6 +196,27 @@ def fused_router_topk(hidden_states, router_weight, correction_bias, topk: int,
     r = biased_grouped_topk(logits, correction_bias, topk, renormalize, num_expert_group,
                             topk_group, routed_scaling_factor, lib=lib)
     return r, logits
+
+
+def softcap_logits(logits, softcap: float, lib=None) -> np.ndarray:
+    """c * tanh(logits / c) elementwise (oracle_softcap); c == 0 returns a copy."""
+    x = as_f64(logits)
+    out = np.empty_like(x)
+    lib = lib or load()
+    if lib.oracle_softcap(_ptr(x, _DBL), x.size, float(softcap), _ptr(out, _DBL)) != 0:
+        raise ValueError("oracle_softcap: invalid arguments")
+    return out
+
+
+def fused_router_top1(hidden_states, router_weight, softcap: float = 0.0, weight_layout: int = 0,
+                      lib=None):
+    """The fused router's top-1 form: projection, softcapping (c == 0: none),
+    then softmax top-1 without renormalisation, so the weight is the softmax
+    probability of the arg-max, 1 / sum_e exp(l_e - max l).  Returns
+    (Routing, capped logits)."""
+    logits = router_logits(hidden_states, router_weight, weight_layout=weight_layout, lib=lib)
+    capped = softcap_logits(logits, softcap, lib=lib)
+    return topk_softmax(capped, 1, False, lib=lib), capped
 
 
 class Permutation:

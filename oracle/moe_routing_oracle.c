@@ -8,7 +8,8 @@
  *
  * Style: one row at a time, one step at a time, in double precision, in the
  * order the pages give the steps.  The only library primitives used are
- * exp() and qsort().  There is deliberately no blocking, fusion or cleverness.
+ * exp(), tanh() and qsort().  There is deliberately no blocking, fusion or
+ * cleverness.
  *
  * Sources (pages on SGLang MoE routing; cited by page title and section):
  *   [M] "MiniMax-M3 모델을 위한 FP8 Attention GEMM 최적화 및 성능 개선"
@@ -23,7 +24,8 @@
  *                                   the choice, group score = sum of the top-2
  *                                   biased scores in the group
  *       §5 Fused MoE Router       - logits = hidden_states x router weight in
- *                                   fp32 accumulation, routing on the result
+ *                                   fp32 accumulation, optional softcapping
+ *                                   c * tanh(logits / c), routing on the result
  *       §6 공유 전문가 슬롯 할당       - the last slot goes to a shared expert
  *   [A] "[sglang] SGLang MoE 라우팅 최적화: AMD GPU에서 aiter.biased_grouped_topk 활용"
  *       코드 분석 (After)           - sigmoid + correction_bias routing expressed
@@ -254,6 +256,23 @@ int oracle_router_logits(const double* h, const double* w, int64_t M, int K, int
             }
             logits[i * (int64_t)E + e] = acc;
         }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * oracle_softcap: the logit softcapping of [R] §5 (the fused router's
+ * Softcapping step), out[i] = c * tanh(x[i] / c) for n values.  The page
+ * applies it only when the softcapping constant is nonzero; c == 0 copies the
+ * values unchanged.  x and out may be the same array.
+ * ------------------------------------------------------------------------- */
+int oracle_softcap(const double* x, int64_t n, double c, double* out) {
+    if (n < 0 || c != c || c < 0.0) return ORACLE_BAD_ARGS;
+    for (int64_t i = 0; i < n; ++i) {
+        if (c == 0.0)
+            out[i] = x[i];
+        else
+            out[i] = c * tanh(x[i] / c);
     }
     return ORACLE_OK;
 }

@@ -16,7 +16,12 @@ Pins used:
 * the router projection against numpy's float64 matmul and a hand case;
 * the expert permutation against a hand case, and against numpy's stable
   argsort, bincount and cumsum on random and routed ids (plus its inverse-
-  permutation and stability invariants).
+  permutation and stability invariants);
+* softcapping against the closed form tanh(ln(a) / 2) = (a - 1) / (a + 1), its
+  saturation at +-c and the identity at c = 0;
+* the fused router's top-1 form against hand cases whose weight is the
+  logistic function of the logit gap, and against numpy's arg-max and the
+  page's 1 / sum exp(l - max l) on random rows.
 """
 from __future__ import annotations
 
@@ -299,8 +304,65 @@ def check_postprocess(lib) -> list[str]:
     return fails
 
 
+def check_softcap(lib) -> list[str]:
+    """c * tanh(x / c) at points where tanh has a closed form: x = (c / 2) ln a
+    gives c (a - 1) / (a + 1).  Also saturation and the c = 0 identity."""
+    fails = []
+    for c in (0.5, 1.0, 4.0, 30.0):
+        a = np.array([1.0 / 1024, 0.25, 1.0 / 3, 1.0, 1.5, 3.0, 7.0, 1e6])
+        x = (c / 2.0) * np.log(a)
+        want = c * (a - 1.0) / (a + 1.0)
+        got = oracle.softcap_logits(x, c, lib=lib)
+        if not np.allclose(got, want, rtol=1e-14, atol=1e-15 * c):
+            fails.append(f"softcap c={c}: {got.tolist()} != {want.tolist()}")
+        big = oracle.softcap_logits(np.array([60.0 * c, -60.0 * c]), c, lib=lib)
+        if not np.allclose(big, [c, -c], rtol=1e-15, atol=0):
+            fails.append(f"softcap c={c} does not saturate at +-c: {big.tolist()}")
+    x = np.random.default_rng(3).standard_normal(50) * 20
+    if not np.array_equal(oracle.softcap_logits(x, 0.0, lib=lib), x):
+        fails.append("softcap with c = 0 changed the logits")
+    return fails
+
+
+def check_fused_top1(lib) -> list[str]:
+    """Hand cases (tests/golden/fused_top1_small.json) and random rows."""
+    doc = json.load(open(os.path.join(GOLDEN, "fused_top1_small.json")))
+    fails = []
+    for case in doc["cases"]:
+        if "hidden" in case:
+            h = np.asarray(case["hidden"], np.float64)
+        else:
+            h = 2.0 * np.log(np.asarray(case["a"], np.float64))
+        w = np.asarray(case["weight_ke"], np.float64)
+        r, capped = oracle.fused_router_top1(h, w, case["softcap"], lib=lib)
+        want_w = [1.0 / (1.0 + math.exp(-d)) for d in case["gap"]]
+        if r.ids[:, 0].tolist() != case["ids"]:
+            fails.append(f"fused top-1 {case['name']}: ids {r.ids[:, 0].tolist()} != {case['ids']}")
+        if not np.allclose(r.weights[:, 0], want_w, rtol=0, atol=1e-12):
+            fails.append(f"fused top-1 {case['name']}: weights {r.weights[:, 0].tolist()} != {want_w}")
+        if "capped" in case and not np.allclose(capped, case["capped"], rtol=0, atol=1e-12):
+            fails.append(f"fused top-1 {case['name']}: capped logits {capped.tolist()}")
+    # random rows: arg-max (first of equals) and the page's invsumexp weight
+    rng = np.random.default_rng(29)
+    h = rng.standard_normal((40, 24))
+    wt = rng.standard_normal((24, 8)) * 0.5
+    for c in (0.0, 2.0, 30.0):
+        r, capped = oracle.fused_router_top1(h, wt, c, lib=lib)
+        l = h @ wt
+        if not np.array_equal(r.ids[:, 0], np.argmax(l, axis=1)):
+            fails.append(f"fused top-1 c={c}: arg-max differs from numpy's")
+        inv = 1.0 / np.sum(np.exp(capped - capped.max(axis=1, keepdims=True)), axis=1)
+        if not np.allclose(r.weights[:, 0], inv, rtol=1e-13, atol=0):
+            fails.append(f"fused top-1 c={c}: weight is not 1 / sum exp(l - max l)")
+        r_t, _ = oracle.fused_router_top1(h, np.ascontiguousarray(wt.T), c, weight_layout=1, lib=lib)
+        if not np.array_equal(r_t.ids, r.ids) or not np.allclose(r_t.weights, r.weights, rtol=1e-14, atol=0):
+            fails.append(f"fused top-1 c={c}: (E, K) weight layout differs from (K, E)")
+    return fails
+
+
 ALL_CHECKS = (check_golden, check_router_golden, check_router_numpy, check_brute, check_library,
-              check_permutation_golden, check_permutation_numpy, check_postprocess)
+              check_permutation_golden, check_permutation_numpy, check_postprocess, check_softcap,
+              check_fused_top1)
 
 
 def run_all(lib) -> list[str]:

@@ -38,7 +38,9 @@ def test_fill_shared_expert_slot(M, k, rsf):
     assert np.array_equal(ids.cpu().numpy(), ids_ref)
     got = w.cpu().numpy().astype(np.float64)
     assert np.array_equal(got[:, :-1], w0[:, :-1].astype(np.float64))       # other slots untouched
-    assert np.allclose(got[:, -1], w_ref[:, -1], rtol=1e-6, atol=0.0)
+    # the kernel sums the k-1 positive fp32 weights in order and divides once:
+    # at most (k-2) + 1 roundings of 2^-24 relative to the sum
+    assert np.allclose(got[:, -1], w_ref[:, -1], rtol=max(k - 1, 1) * 2.0**-24, atol=0.0)
 
 
 @pytest.mark.parametrize("M,k", [(1, 8), (5000, 8), (16384, 9), (700, 1), (129, 32)])

@@ -255,15 +255,15 @@ def test_aiter_variant_is_the_plain_call_for_fp32_logits():
                                                (700, 64, 8, 3, 5, True)])     # generic kernel
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_softcapped_softmax(M, E, G, TG, k, renorm, dtype):
-    """moe_grouped_topk_softcap: the oracle's softmax routing of the capped
-    logits 30 * tanh(x / 30) (computed in double).  Weight tolerance for fp32
+    """moe_grouped_topk_softcap: the oracle's softmax routing of the oracle's
+    capped logits 30 * tanh(x / 30) (computed in double).  Weight tolerance for fp32
     logits: tanhf's ~2 ulp, times c, plus roundings, gives ~4e-7 * c on each
     capped logit and, through exp and the sum, below 1.4e-5 relative; 2e-5."""
     c = 30.0
     x = inputs.random_logits(M, E, 20.0, dtype, seed=E + k + M)
     w, ids = moe.grouped_topk(x.to(DEV), k, renorm, G, TG, 1.5, softcap=c)
     torch.cuda.synchronize()
-    xc = c * np.tanh(oracle.as_f64(x) / c)
+    xc = oracle.softcap_logits(x, c)
     orc = oracle.grouped_topk(xc, k, renorm, G, TG, 1.5)
     rep = parity.compare(w.cpu().numpy(), ids.cpu().numpy(), orc, E=E, G=G, TG=TG, k=k, renorm=renorm, rsf=1.5,
                          fp32_logits=(dtype == torch.float32),

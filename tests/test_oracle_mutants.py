@@ -47,6 +47,9 @@ MUTANTS = {
                                 "weights[i * (int64_t)k + (k - 1)] = sum * rsf;"),
     "shared_id_offset": ("ids[i * (int64_t)k + (k - 1)] = E + pick[i];", "ids[i * (int64_t)k + (k - 1)] = pick[i];"),
     "sort_unstable": ("while (b >= 0 && id[b] > ka) {", "while (b >= 0 && id[b] >= ka) {"),
+    "softcap_unscaled": ("out[i] = c * tanh(x[i] / c);", "out[i] = tanh(x[i] / c);"),
+    "softcap_times_inside": ("out[i] = c * tanh(x[i] / c);", "out[i] = c * tanh(x[i] * c);"),
+    "softcap_zero_clears": ("            out[i] = x[i];\n", "            out[i] = 0.0;\n"),
 }
 
 
