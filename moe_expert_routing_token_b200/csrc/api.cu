@@ -266,6 +266,7 @@ int route(const void* logits, int dtype, const float* bias, int64_t M, int E, in
     if (K < 1 || K > TG * (E / G))
         return fail(MOE_ERR_INVALID_ARG, "%s: topk=%d outside [1, topk_group*E/G=%d]", who, K, TG * (E / G));
     if (!std::isfinite(rsf)) return fail(MOE_ERR_INVALID_ARG, "%s: routed_scaling_factor is not finite", who);
+    if (!std::isfinite(softcap)) return fail(MOE_ERR_INVALID_ARG, "%s: softcap is not finite", who);
     if (E > 1024) return fail(MOE_ERR_UNSUPPORTED, "%s: E=%d > 1024", who, E);
     if (K > 32) return fail(MOE_ERR_UNSUPPORTED, "%s: topk=%d > 32", who, K);
     if (M == 0) return MOE_OK;
@@ -288,7 +289,6 @@ int route(const void* logits, int dtype, const float* bias, int64_t M, int E, in
     a.weights = weights;
     a.ids = ids;
     a.bias_bf16 = (bias_bf16 && dtype == MOE_DTYPE_BF16) ? 1 : 0;  // an fp32 cast of fp32 logits changes nothing
-    if (!std::isfinite(softcap)) return fail(MOE_ERR_INVALID_ARG, "%s: softcap is not finite", who);
     a.softcap = (scoring == kSoftmax) ? softcap : 0.0f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 

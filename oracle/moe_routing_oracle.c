@@ -264,10 +264,11 @@ int oracle_router_logits(const double* h, const double* w, int64_t M, int K, int
  * oracle_softcap: the logit softcapping of [R] §5 (the fused router's
  * Softcapping step), out[i] = c * tanh(x[i] / c) for n values.  The page
  * applies it only when the softcapping constant is nonzero; c == 0 copies the
- * values unchanged.  x and out may be the same array.
+ * values unchanged.  c and -c give the same values (tanh is odd); c must be
+ * finite.  x and out may be the same array.
  * ------------------------------------------------------------------------- */
 int oracle_softcap(const double* x, int64_t n, double c, double* out) {
-    if (n < 0 || c != c || c < 0.0) return ORACLE_BAD_ARGS;
+    if (n < 0 || c != c || c == INFINITY || c == -INFINITY) return ORACLE_BAD_ARGS;
     for (int64_t i = 0; i < n; ++i) {
         if (c == 0.0)
             out[i] = x[i];

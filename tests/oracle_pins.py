@@ -321,6 +321,8 @@ def check_softcap(lib) -> list[str]:
     x = np.random.default_rng(3).standard_normal(50) * 20
     if not np.array_equal(oracle.softcap_logits(x, 0.0, lib=lib), x):
         fails.append("softcap with c = 0 changed the logits")
+    if not np.array_equal(oracle.softcap_logits(x, -4.0, lib=lib), oracle.softcap_logits(x, 4.0, lib=lib)):
+        fails.append("softcap with -c differs from c")
     return fails
 
 

@@ -75,6 +75,15 @@ def test_empty_batch_is_ok_without_launch(lib):
     assert lib.moe_biased_grouped_topk(None, 1, None, 0, 256, 8, 1, 8, 4, 2.5, None, None, None) == 0
 
 
+def test_softcap_validation(lib):
+    # moe_grouped_topk_softcap(logits, dtype, M, E, topk, renorm, G, TG, rsf, softcap, w, ids, stream)
+    for c in (float("nan"), float("inf"), -float("inf")):
+        for M in (4, 0):                                  # rejected even for an empty batch
+            assert lib.moe_grouped_topk_softcap(P, 0, M, 8, 2, 1, 4, 2, 1.0, c, P, P, None) == 1
+            assert b"softcap" in lib.moe_last_error()
+    assert lib.moe_grouped_topk_softcap(None, 0, 0, 8, 2, 1, 4, 2, 1.0, 30.0, None, None, None) == 0
+
+
 def test_biased_validation(lib):
     # bias pointer not 4-byte aligned
     assert lib.moe_biased_grouped_topk(P, 1, P + 1, 4, 256, 8, 1, 8, 4, 2.5, P, P, None) == 1
