@@ -206,6 +206,7 @@ MOE_API size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E);
  *   router_weight   device, bf16, (K, E) if weight_layout == MOE_WEIGHT_K_BY_E
  *                   or (E, K) if MOE_WEIGHT_E_BY_K
  *   correction_bias device, (E,) fp32, or NULL
+ *   M               tokens, below 2^31 (else MOE_ERR_UNSUPPORTED)
  *   K               hidden size, a positive multiple of 64
  *   E               experts; the fused router is built for E == 256
  *   logits_out      device, (M, E) fp32 out, or NULL (debug: the fp32 logits

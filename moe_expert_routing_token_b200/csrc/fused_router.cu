@@ -668,6 +668,10 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
         snprintf(msg, sizeof msg, "%s: num_expert_group=%d / topk=%d not supported", who, num_expert_group, topk);
         return set_error(MOE_ERR_UNSUPPORTED, msg);
     }
+    if (M >= ((int64_t)1 << 31)) {  // tile counts and the outputs' row index stay within int32 grids
+        snprintf(msg, sizeof msg, "%s: M=%lld >= 2^31", who, (long long)M);
+        return set_error(MOE_ERR_UNSUPPORTED, msg);
+    }
     if (M == 0) return MOE_OK;
     if (!hidden_states || !router_weight || !topk_weights || !topk_ids)
         return set_error(MOE_ERR_INVALID_ARG, "moe_fused_router_topk: null pointer argument");

@@ -198,7 +198,9 @@ extern "C" {
 
 size_t moe_expert_permutation_workspace_size(int64_t M, int32_t k, int32_t E) {
     if (M < 0 || k < 1 || E < 1 || E > moe::kPermMaxE) return (size_t)-1;
+    if (M >= ((int64_t)1 << 31)) return (size_t)-1;  // M * k below: no overflow
     const int64_t n = M * (int64_t)k;
+    if (n >= ((int64_t)1 << 31)) return (size_t)-1;
     return (size_t)(moe::perm_tiles(n) * E * (int64_t)sizeof(int32_t));
 }
 
@@ -216,8 +218,9 @@ int moe_expert_permutation(const int32_t* topk_ids, const float* topk_weights, i
         std::snprintf(msg, sizeof msg, "moe_expert_permutation: E=%d > %d", E, kPermMaxE);
         return set_error(MOE_ERR_UNSUPPORTED, msg);
     }
+    if (M >= ((int64_t)1 << 31) || M * (int64_t)k >= ((int64_t)1 << 31))
+        return set_error(MOE_ERR_UNSUPPORTED, "moe_expert_permutation: M*k >= 2^31");
     const int64_t n = M * (int64_t)k;
-    if (n >= ((int64_t)1 << 31)) return set_error(MOE_ERR_UNSUPPORTED, "moe_expert_permutation: M*k >= 2^31");
     if (!expert_counts || !expert_offsets)
         return set_error(MOE_ERR_INVALID_ARG, "moe_expert_permutation: null counts or offsets");
     if (n > 0 && (!topk_ids || !gather_indx || !scatter_indx))

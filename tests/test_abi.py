@@ -96,6 +96,13 @@ def test_fused_router_workspace_query(lib):
     assert n != ctypes.c_size_t(-1).value
 
 
+def test_fused_router_rejects_huge_batches(lib):
+    # (hidden, W, layout, bias, M, K, E, topk, renorm, G, TG, rsf, w, ids, logits_out, ws, ws_bytes, stream)
+    assert lib.moe_fused_router_topk(P, P, 0, None, 1 << 31, 7168, 256, 8, 1, 8, 4, 2.5, P, P, None,
+                                     None, 0, None) == 2
+    assert b"2^31" in lib.moe_last_error()
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(4, 8)
@@ -115,6 +122,11 @@ def test_expert_permutation_validation(lib):
     assert lib.moe_expert_permutation(P, None, 4, 2, 16, P, P, P, P, None, P, 3, None) == 1     # workspace short
     assert b"workspace" in lib.moe_last_error()
     assert lib.moe_expert_permutation(P, None, 4, 2, 16, None, P, P, P, None, P, 4096, None) == 1  # no counts
+    # M*k at or beyond 2^31, including products that overflow int64
+    for M, k in ((1 << 28, 8), (1 << 40, 8), (1 << 62, 32)):
+        assert lib.moe_expert_permutation_workspace_size(M, k, 256) == ctypes.c_size_t(-1).value
+        assert lib.moe_expert_permutation(P, None, M, k, 256, P, P, P, P, None, P, 1 << 40, None) == 2
+        assert b"2^31" in lib.moe_last_error()
 
 
 def test_postprocess_validation(lib):
