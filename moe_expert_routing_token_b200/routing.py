@@ -133,14 +133,27 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _on(device):
+    """Make the operands' device current for the call: the library sizes
+    grids, sets kernel attributes and launches on the current device."""
+    return torch.cuda.device(device)
+
+
+def _same_device(device, **tensors) -> None:
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, not on {device} with the other operands")
+
+
 def topk_softmax(gating_output: torch.Tensor, topk: int, renormalize: bool, out=None):
     """Softmax top-k of each row.  Returns (topk_weights fp32, topk_ids int32)."""
     _cuda_2d(gating_output, "gating_output")
     M, E = gating_output.shape
     w, ids = _outputs(M, topk, gating_output.device, out)
-    st = lib().moe_topk_softmax(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
-                                int(bool(renormalize)), w.data_ptr(), ids.data_ptr(),
-                                _stream(gating_output.device))
+    with _on(gating_output.device):
+        st = lib().moe_topk_softmax(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
+                                    int(bool(renormalize)), w.data_ptr(), ids.data_ptr(),
+                                    _stream(gating_output.device))
     _check(st, "moe_topk_softmax")
     return w, ids
 
@@ -154,16 +167,18 @@ def grouped_topk(gating_output: torch.Tensor, topk: int, renormalize: bool, num_
     M, E = gating_output.shape
     w, ids = _outputs(M, topk, gating_output.device, out)
     if softcap:
-        st = lib().moe_grouped_topk_softcap(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
-                                            int(bool(renormalize)), num_expert_group, topk_group,
-                                            float(routed_scaling_factor), float(softcap), w.data_ptr(),
-                                            ids.data_ptr(), _stream(gating_output.device))
+        with _on(gating_output.device):
+            st = lib().moe_grouped_topk_softcap(gating_output.data_ptr(), _dtype_code(gating_output), M, E,
+                                                topk, int(bool(renormalize)), num_expert_group, topk_group,
+                                                float(routed_scaling_factor), float(softcap), w.data_ptr(),
+                                                ids.data_ptr(), _stream(gating_output.device))
         _check(st, "moe_grouped_topk_softcap")
         return w, ids
-    st = lib().moe_grouped_topk(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
-                                int(bool(renormalize)), num_expert_group, topk_group,
-                                float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
-                                _stream(gating_output.device))
+    with _on(gating_output.device):
+        st = lib().moe_grouped_topk(gating_output.data_ptr(), _dtype_code(gating_output), M, E, topk,
+                                    int(bool(renormalize)), num_expert_group, topk_group,
+                                    float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
+                                    _stream(gating_output.device))
     _check(st, "moe_grouped_topk")
     return w, ids
 
@@ -180,10 +195,11 @@ def biased_grouped_topk(gating_output: torch.Tensor, correction_bias, topk: int,
     bp = _bias_ptr(correction_bias, E, gating_output.device)
     w, ids = _outputs(M, topk, gating_output.device, out)
     fn = lib().moe_biased_grouped_topk_aiter if bias_as_logits_dtype else lib().moe_biased_grouped_topk
-    st = fn(gating_output.data_ptr(), _dtype_code(gating_output), bp, M, E,
-            topk, int(bool(renormalize)), num_expert_group, topk_group,
-            float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
-            _stream(gating_output.device))
+    with _on(gating_output.device):
+        st = fn(gating_output.data_ptr(), _dtype_code(gating_output), bp, M, E,
+                topk, int(bool(renormalize)), num_expert_group, topk_group,
+                float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
+                _stream(gating_output.device))
     _check(st, "moe_biased_grouped_topk")
     return w, ids
 
@@ -225,6 +241,7 @@ def fused_router_topk(hidden_states: torch.Tensor, router_weight: torch.Tensor, 
     if Kw != K:
         raise ValueError("router_weight does not match hidden_states' hidden size")
     dev = hidden_states.device
+    _same_device(dev, router_weight=router_weight, workspace=workspace)
     bp = _bias_ptr(correction_bias, E, dev)
     w, ids = _outputs(M, topk, dev, out)
     logits = torch.empty(M, E, dtype=torch.float32, device=dev) if return_logits else None
@@ -233,11 +250,12 @@ def fused_router_topk(hidden_states: torch.Tensor, router_weight: torch.Tensor, 
         # the workspace must start zeroed; the library leaves it zeroed again
         workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
     wsp = workspace.data_ptr() if (need and workspace is not None) else None
-    st = lib().moe_fused_router_topk(hidden_states.data_ptr(), router_weight.data_ptr(), layout, bp, M,
-                                     K, E, topk, int(bool(renormalize)), num_expert_group, topk_group,
-                                     float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
-                                     None if logits is None else logits.data_ptr(), wsp,
-                                     need if wsp else 0, _stream(dev))
+    with _on(dev):
+        st = lib().moe_fused_router_topk(hidden_states.data_ptr(), router_weight.data_ptr(), layout, bp, M,
+                                         K, E, topk, int(bool(renormalize)), num_expert_group, topk_group,
+                                         float(routed_scaling_factor), w.data_ptr(), ids.data_ptr(),
+                                         None if logits is None else logits.data_ptr(), wsp,
+                                         need if wsp else 0, _stream(dev))
     _check(st, "moe_fused_router_topk")
     return (w, ids, logits) if return_logits else (w, ids)
 
@@ -264,6 +282,7 @@ def expert_permutation(topk_ids: torch.Tensor, num_experts: int, topk_weights=No
         _cuda_2d(topk_weights, "topk_weights")
         if topk_weights.dtype != torch.float32 or tuple(topk_weights.shape) != (M, k):
             raise ValueError("topk_weights must be fp32 with the shape of topk_ids")
+    _same_device(dev, topk_weights=topk_weights, workspace=workspace)
     need = expert_permutation_workspace_size(M, k, num_experts)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
@@ -272,11 +291,13 @@ def expert_permutation(topk_ids: torch.Tensor, num_experts: int, topk_weights=No
     gather = torch.empty(n, dtype=torch.int32, device=dev)
     scatter = torch.empty(n, dtype=torch.int32, device=dev)
     gate = None if topk_weights is None else torch.empty(n, dtype=torch.float32, device=dev)
-    _check(lib().moe_expert_permutation(
-        topk_ids.data_ptr(), None if topk_weights is None else topk_weights.data_ptr(), M, k, int(num_experts),
-        counts.data_ptr(), offsets.data_ptr(), gather.data_ptr(), scatter.data_ptr(),
-        None if gate is None else gate.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(dev)),
-        "moe_expert_permutation")
+    with _on(dev):
+        st = lib().moe_expert_permutation(
+            topk_ids.data_ptr(), None if topk_weights is None else topk_weights.data_ptr(), M, k,
+            int(num_experts), counts.data_ptr(), offsets.data_ptr(), gather.data_ptr(), scatter.data_ptr(),
+            None if gate is None else gate.data_ptr(), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(st, "moe_expert_permutation")
     return counts, offsets, gather, scatter, gate
 
 
@@ -286,6 +307,7 @@ def _result_pair(topk_weights: torch.Tensor, topk_ids: torch.Tensor):
     if topk_weights.dtype != torch.float32 or topk_ids.dtype != torch.int32 or \
             topk_weights.shape != topk_ids.shape:
         raise ValueError("topk_weights must be fp32 and topk_ids int32 of the same (M, k) shape")
+    _same_device(topk_ids.device, topk_weights=topk_weights)
     return topk_ids.shape
 
 
@@ -298,18 +320,23 @@ def fill_shared_expert_slot(topk_weights: torch.Tensor, topk_ids: torch.Tensor, 
     if not shared_pick.is_cuda or shared_pick.dtype != torch.int32 or shared_pick.numel() != M or \
             not shared_pick.is_contiguous():
         raise ValueError("shared_pick must be a contiguous CUDA int32 tensor of M values")
+    _same_device(topk_ids.device, shared_pick=shared_pick)
     rsf = 0.0 if routed_scaling_factor is None else float(routed_scaling_factor)
     if routed_scaling_factor is not None and rsf == 0.0:
         raise ValueError("routed_scaling_factor 0 is reserved for None")
-    _check(lib().moe_fill_shared_expert_slot(topk_weights.data_ptr(), topk_ids.data_ptr(), M, k, int(num_experts),
-                                             int(num_shared), shared_pick.data_ptr(), rsf,
-                                             _stream(topk_ids.device)), "moe_fill_shared_expert_slot")
+    with _on(topk_ids.device):
+        st = lib().moe_fill_shared_expert_slot(topk_weights.data_ptr(), topk_ids.data_ptr(), M, k,
+                                               int(num_experts), int(num_shared), shared_pick.data_ptr(), rsf,
+                                               _stream(topk_ids.device))
+    _check(st, "moe_fill_shared_expert_slot")
     return topk_weights, topk_ids
 
 
 def sort_topk_by_id(topk_weights: torch.Tensor, topk_ids: torch.Tensor):
     """In place: each row's (weight, id) pairs in ascending id (stable)."""
     M, k = _result_pair(topk_weights, topk_ids)
-    _check(lib().moe_sort_topk_by_id(topk_weights.data_ptr(), topk_ids.data_ptr(), M, k,
-                                     _stream(topk_ids.device)), "moe_sort_topk_by_id")
+    with _on(topk_ids.device):
+        st = lib().moe_sort_topk_by_id(topk_weights.data_ptr(), topk_ids.data_ptr(), M, k,
+                                       _stream(topk_ids.device))
+    _check(st, "moe_sort_topk_by_id")
     return topk_weights, topk_ids
