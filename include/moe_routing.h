@@ -58,8 +58,9 @@ extern "C" {
 /* 1: the routing calls and the fused router.  2: adds the allocation-free
  * fused router, the softcap and aiter variants, the expert permutation, the
  * shared-expert slot, the ascending-id order and the bounded-wait self-test
- * (every version-1 call keeps its signature and meaning). */
-#define MOE_ROUTING_ABI_VERSION 2
+ * (every version-1 call keeps its signature and meaning).  3: adds the
+ * small-E top-1 router moe_fused_router_top1 (earlier calls unchanged). */
+#define MOE_ROUTING_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -267,6 +268,37 @@ MOE_API int moe_fused_router_topk_noalloc(const void* hidden_states, const void*
                                           int32_t num_expert_group, int32_t topk_group,
                                           float routed_scaling_factor, float* topk_weights,
                                           int32_t* topk_ids, float* logits_out, void* stream);
+
+/*
+ * moe_fused_router_top1 - the CUDA-core fused router of [R] §5 for small
+ * expert counts: per token row,
+ *     l_e = sum_k h[k] * W(k, e)              (bf16 inputs, fp32 sums)
+ *     id  = arg-max_e l_e                     (lower index among equal logits)
+ *     w   = 1 / sum_e exp(cap(l_e) - cap(l_id)),  cap(x) = softcap * tanh(x / softcap)
+ * i.e. softcapping (when softcap != 0; 0 = none), then top-1 with the
+ * softmax probability of the chosen expert as its weight (the page's
+ * invsumexp).  cap is strictly increasing, so the arg-max of the raw logits
+ * is the arg-max of the capped ones.
+ *
+ *   hidden_states   device, (M, K) bf16, 16-byte aligned
+ *   router_weight   device, bf16, (K, E) if weight_layout == MOE_WEIGHT_K_BY_E
+ *                   or (E, K) if MOE_WEIGHT_E_BY_K (the page's layout),
+ *                   16-byte aligned
+ *   K               hidden size, a positive multiple of 8
+ *   E               experts, 1..8 (else MOE_ERR_UNSUPPORTED); the page sends
+ *                   E > 8 to its tensor-core kernel
+ *   softcap         finite; 0 = no softcapping; c and -c give the same result
+ *   topk_weights    device, (M, 1) fp32 out
+ *   topk_ids        device, (M, 1) int32 out
+ *   logits_out      device, (M, E) fp32 out, or NULL (debug: the raw logits)
+ * Every batch size runs on the CUDA cores: at E <= 8 the projection does at
+ * most 8 flops per byte of hidden state, so it streams at HBM bandwidth (the
+ * page's batch-size switch to tensor cores has no counterpart here).
+ * Asynchronous on `stream`; no allocation; M == 0 launches nothing.
+ */
+MOE_API int moe_fused_router_top1(const void* hidden_states, const void* router_weight, int weight_layout,
+                                  int64_t M, int32_t K, int32_t E, float softcap, float* topk_weights,
+                                  int32_t* topk_ids, float* logits_out, void* stream);
 
 /*
  * moe_expert_permutation - the expert-sorted token permutation that follows

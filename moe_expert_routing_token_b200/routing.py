@@ -50,6 +50,8 @@ SIGNATURES = {
                                              _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_fused_router_topk_noalloc": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _vp, _i64, _i32, _i32, _i32,
                                                      _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
+    "moe_fused_router_top1": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _i64, _i32, _i32, _f32, _vp, _vp, _vp,
+                                             _vp]),
     "moe_expert_permutation_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_fill_shared_expert_slot": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _i32, _vp, _f32, _vp]),
     "moe_sort_topk_by_id": (ctypes.c_int, [_vp, _vp, _i64, _i32, _vp]),
@@ -257,6 +259,37 @@ def fused_router_topk(hidden_states: torch.Tensor, router_weight: torch.Tensor, 
                                          None if logits is None else logits.data_ptr(), wsp,
                                          need if wsp else 0, _stream(dev))
     _check(st, "moe_fused_router_topk")
+    return (w, ids, logits) if return_logits else (w, ids)
+
+
+def fused_router_top1(hidden_states: torch.Tensor, router_weight: torch.Tensor, softcap: float = 0.0,
+                      weight_layout: str = "ek", return_logits: bool = False, out=None):
+    """Router projection, softcapping and top-1 on the CUDA cores, for E <= 8
+    experts (moe_fused_router_top1).  ``weight_layout`` "ek": router_weight
+    is (E, K); "ke": (K, E).  Returns (weights (M, 1) fp32, ids (M, 1) int32)
+    or, with ``return_logits``, also the raw fp32 logits (M, E)."""
+    _cuda_2d(hidden_states, "hidden_states")
+    _cuda_2d(router_weight, "router_weight")
+    if hidden_states.dtype != torch.bfloat16 or router_weight.dtype != torch.bfloat16:
+        raise ValueError("hidden_states and router_weight must be bfloat16")
+    M, K = hidden_states.shape
+    if weight_layout == "ek":
+        layout, (E, Kw) = MOE_WEIGHT_E_BY_K, router_weight.shape
+    elif weight_layout == "ke":
+        layout, (Kw, E) = MOE_WEIGHT_K_BY_E, router_weight.shape
+    else:
+        raise ValueError("weight_layout must be 'ek' or 'ke'")
+    if Kw != K:
+        raise ValueError("router_weight does not match hidden_states' hidden size")
+    dev = hidden_states.device
+    _same_device(dev, router_weight=router_weight)
+    w, ids = _outputs(M, 1, dev, out)
+    logits = torch.empty(M, E, dtype=torch.float32, device=dev) if return_logits else None
+    with _on(dev):
+        st = lib().moe_fused_router_top1(hidden_states.data_ptr(), router_weight.data_ptr(), layout, M, K, E,
+                                         float(softcap), w.data_ptr(), ids.data_ptr(),
+                                         None if logits is None else logits.data_ptr(), _stream(dev))
+    _check(st, "moe_fused_router_top1")
     return (w, ids, logits) if return_logits else (w, ids)
 
 

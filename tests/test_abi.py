@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 2
+    assert lib.moe_abi_version() == 3
     assert lib.moe_status_string(0) == b"MOE_OK"
     assert lib.moe_status_string(1) == b"MOE_ERR_INVALID_ARG"
     assert lib.moe_status_string(2) == b"MOE_ERR_UNSUPPORTED"
@@ -101,6 +101,22 @@ def test_fused_router_rejects_huge_batches(lib):
     assert lib.moe_fused_router_topk(P, P, 0, None, 1 << 31, 7168, 256, 8, 1, 8, 4, 2.5, P, P, None,
                                      None, 0, None) == 2
     assert b"2^31" in lib.moe_last_error()
+
+
+def test_top1_router_validation(lib):
+    # (hidden, W, layout, M, K, E, softcap, w, ids, logits_out, stream)
+    assert lib.moe_fused_router_top1(P, P, 1, -1, 64, 8, 0.0, P, P, None, None) == 1      # M < 0
+    assert lib.moe_fused_router_top1(P, P, 1, 4, 0, 8, 0.0, P, P, None, None) == 1        # K < 1
+    assert lib.moe_fused_router_top1(P, P, 2, 4, 64, 8, 0.0, P, P, None, None) == 1       # layout
+    assert lib.moe_fused_router_top1(P, P, 1, 4, 64, 8, float("nan"), P, P, None, None) == 1
+    assert b"softcap" in lib.moe_last_error()
+    assert lib.moe_fused_router_top1(P, P, 1, 4, 64, 9, 0.0, P, P, None, None) == 2       # E > 8
+    assert b"E <= 8" in lib.moe_last_error()
+    assert lib.moe_fused_router_top1(P, P, 1, 4, 60, 8, 0.0, P, P, None, None) == 2       # K % 8
+    assert lib.moe_fused_router_top1(None, P, 1, 4, 64, 8, 0.0, P, P, None, None) == 1    # null
+    assert lib.moe_fused_router_top1(P + 8, P, 1, 4, 64, 8, 0.0, P, P, None, None) == 1   # 16-B alignment
+    assert b"aligned" in lib.moe_last_error()
+    assert lib.moe_fused_router_top1(None, None, 0, 0, 64, 8, 30.0, None, None, None, None) == 0  # empty
 
 
 def test_binding_rejects_cpu_tensors():

@@ -1,0 +1,136 @@
+"""The CUDA-core top-1 router (projection, softcapping, top-1 with the softmax
+weight 1 / sum exp(cap(l) - cap(l_max))) against the CPU oracle, through the
+C ABI (GPU only).
+
+Three checks per case:
+* the kernel's raw fp32 logits (debug output) against the oracle's double
+  projection, within the fp32 summation bound below;
+* the top-1 of those logits against the oracle fed the same logits (softcap
+  and weight in double): clear rows need the same id, near-tie rows a valid
+  one; weights within 2e-5 relative;
+* against the oracle's end-to-end result (double projection), with the
+  near-tie margin and the weight tolerance widened by the logits' error.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_expert_routing_token_b200 as moe
+import oracle
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+# Weight tolerance on the kernel's own logits: the capped logit carries
+# tanhf's error (a few ulp of c), the exponent difference twice that, and the
+# base-2 exponential, the E-term sum and the division add a few ulp each:
+# below 1.4e-5 relative at c = 30.
+W_RTOL = 2e-5
+
+
+def _logit_rel(K: int) -> float:
+    """fp32 summation bound for one logit, as a multiple of sum_k |h_k w_k|:
+    each thread chains the FMAs of its ceil(K / 1024) chunks of 8 values,
+    then 5 shuffle levels and 3 cross-warp additions (products of bf16 values
+    are exact in fp32); 16 extra roundings of margin."""
+    per_thread = -(-K // 1024) * 8
+    return (per_thread + 5 + 3 + 16) * 2.0 ** -24
+
+
+def _draw(M, K, E, seed):
+    g = torch.Generator().manual_seed(seed)
+    h = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    w_ek = (torch.randn(E, K, generator=g) * 0.02).to(torch.bfloat16)
+    return h, w_ek
+
+
+def _run(h, w_ek, layout, c):
+    wd = (w_ek if layout == "ek" else w_ek.t().contiguous()).to(DEV)
+    w, ids, logits = moe.fused_router_top1(h.to(DEV), wd, c, weight_layout=layout, return_logits=True)
+    torch.cuda.synchronize()
+    return w.cpu(), ids.cpu(), logits.cpu()
+
+
+def _check(h, w_ek, layout, c):
+    M, K = h.shape
+    E = w_ek.shape[0]
+    w_gpu, ids_gpu, logits_gpu = _run(h, w_ek, layout, c)
+    assert w_gpu.shape == (M, 1) and ids_gpu.shape == (M, 1)
+    ref = oracle.router_logits(h, w_ek, weight_layout=1)
+    absum = np.abs(oracle.as_f64(h)) @ np.abs(oracle.as_f64(w_ek)).T
+    err = np.abs(logits_gpu.double().numpy() - ref)
+    assert np.all(err <= _logit_rel(K) * absum + 1e-30), f"logits max err {err.max():.3g}"
+    # the top-1 step alone: the oracle on the kernel's logits
+    orc_same = oracle.topk_softmax(oracle.softcap_logits(logits_gpu, c), 1, False)
+    rep = parity.compare(w_gpu.numpy(), ids_gpu.numpy(), orc_same, E=E, G=1, TG=1, k=1, renorm=False, rsf=1.0,
+                         fp32_logits=True, w_rtol=W_RTOL)
+    assert rep.ok(), "top-1 of kernel logits: " + rep.summary()
+    # end to end: a logit error e moves each softmax probability by at most
+    # e / 2 (the cap's slope is <= 1) and its logarithm by at most 2 e
+    orc, _ = oracle.fused_router_top1(h, w_ek, c, weight_layout=1)
+    e = float(err.max())
+    rep2 = parity.compare(w_gpu.numpy(), ids_gpu.numpy(), orc, E=E, G=1, TG=1, k=1, renorm=False, rsf=1.0,
+                          fp32_logits=True, eps=parity.EPS + 2 * e, w_rtol=W_RTOL + 4 * e)
+    assert rep2.ok(), "end to end: " + rep2.summary()
+    return rep2
+
+
+@pytest.mark.parametrize("M,K,E,layout,c", [
+    (1, 64, 8, "ek", 0.0),         # one row, 8 of 128 threads carry a chunk
+    (7, 7168, 8, "ek", 30.0),      # a ragged 4-row tile
+    (64, 4096, 8, "ke", 0.0),
+    (511, 2048, 4, "ek", 30.0),    # below the page's 512-token switch
+    (512, 2048, 2, "ke", 2.0),     # at it (here the same kernel)
+    (3000, 7168, 8, "ek", 30.0),   # more tiles than resident blocks
+    (2049, 1032, 3, "ke", 5.0),    # 129 chunks: one thread takes two
+    (100, 512, 1, "ek", 0.0),      # one expert: id 0, weight 1
+])
+def test_top1_router(M, K, E, layout, c):
+    h, w = _draw(M, K, E, seed=M + K + E)
+    _check(h, w, layout, c)
+
+
+@pytest.mark.parametrize("E", [5, 6, 7])
+@pytest.mark.parametrize("layout", ["ek", "ke"])
+def test_every_expert_count(E, layout):
+    h, w = _draw(777, 2048, E, seed=E)
+    _check(h, w, layout, 10.0)
+
+
+def test_zero_rows_and_equal_logits():
+    """A zero hidden row gives equal logits: expert 0, weight 1/E.  Two
+    identical weight rows give two equal largest logits: the lower index."""
+    M, K, E = 256, 1024, 8
+    g = torch.Generator().manual_seed(4)
+    h = torch.randn(M, K, generator=g).abs().to(torch.bfloat16)
+    h[::3] = 0
+    w = torch.zeros(E, K)
+    v = torch.rand(K, generator=g) * 0.05
+    w[2] = v
+    w[5] = v
+    w = w.to(torch.bfloat16)
+    for layout in ("ek", "ke"):
+        wt, ids, logits = _run(h, w, layout, 30.0)
+        zero = np.arange(M) % 3 == 0
+        assert np.all(ids.numpy()[zero, 0] == 0)
+        assert np.allclose(wt.numpy()[zero, 0], 1.0 / E, rtol=1e-6, atol=0)
+        assert np.all(ids.numpy()[~zero, 0] == 2)
+        assert torch.equal(logits[:, 2], logits[:, 5])
+        _check(h, w, layout, 30.0)
+
+
+def test_empty_batch():
+    h = torch.empty(0, 512, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(8, 512, dtype=torch.bfloat16, device=DEV)
+    wt, ids = moe.fused_router_top1(h, w, 30.0)
+    assert wt.shape == (0, 1) and ids.shape == (0, 1)
+
+
+def test_unsupported_shapes_raise():
+    h = torch.zeros(4, 512, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(NotImplementedError, match="E <= 8"):
+        moe.fused_router_top1(h, torch.zeros(16, 512, dtype=torch.bfloat16, device=DEV))
+    with pytest.raises(NotImplementedError, match="multiple of 8"):
+        moe.fused_router_top1(torch.zeros(4, 500, dtype=torch.bfloat16, device=DEV),
+                              torch.zeros(8, 500, dtype=torch.bfloat16, device=DEV))
