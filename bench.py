@@ -46,7 +46,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=480)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="sigmoid",
-                    choices=["sigmoid", "biased", "grouped", "softmax", "fused", "permute"])
+                    choices=["sigmoid", "biased", "grouped", "softmax", "fused", "top1", "permute"])
     ap.add_argument("--M", type=int, default=None, help="tokens per step (default: workload's)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -55,7 +55,8 @@ def parse_args():
     return ap.parse_args()
 
 
-DEFAULT_M = {"sigmoid": 16384, "biased": 4096, "grouped": 16384, "softmax": 64, "fused": 8192, "permute": 16384}
+DEFAULT_M = {"sigmoid": 16384, "biased": 4096, "grouped": 16384, "softmax": 64, "fused": 8192, "top1": 8192,
+             "permute": 16384}
 PERM_K, PERM_E = 8, 256  # the permutation step after the sigmoid workload's routing
 
 
@@ -76,6 +77,11 @@ def workload_desc(name: str, M: int) -> dict:
         d["workload"] = f"softmax grouped top-k DeepSeek-V2 shape, E=160 G=8 TG=3 k=6, M={M}, fp32"
     elif name == "softmax":
         d["workload"] = f"softmax top-k E=8 k=2 renormalise, M={M}, fp32 logits"
+    elif name == "top1":
+        d["workload"] = (f"small-E fused router on the CUDA cores: (M,{sp.K}) bf16 x ({sp.E},{sp.K}) bf16 "
+                         f"weight, softcap {sp.softcap:g}, top-1 with weight 1/sum exp, M={M}")
+        d["K"] = sp.K
+        d["softcap"] = sp.softcap
     else:
         d["workload"] = (f"fused router (M,{sp.K})x({sp.K},{sp.E}) bf16 + biased grouped top-k "
                          f"G=8 TG=4 k=8, M={M}")
@@ -90,7 +96,7 @@ def algorithmic_bytes(name: str, M: int) -> int:
     esz = 2 if str(sp.dtype).endswith("bfloat16") else 4
     out = M * sp.topk * 8
     bias = sp.E * 4 if sp.bias_std is not None else 0
-    if name == "fused":
+    if name in ("fused", "top1"):
         return M * sp.K * 2 + sp.K * sp.E * 2 + out + bias
     return M * sp.E * esz + out + bias
 
@@ -188,6 +194,8 @@ class ClockSampler:
 def oracle_call(name: str, d: dict, rows: slice):
     import oracle
     sp = d["spec"]
+    if name == "top1":
+        return oracle.fused_router_top1(d["hidden"][rows], d["weight"], sp.softcap, weight_layout=1)
     if name == "fused":
         return oracle.fused_router_topk(d["hidden"][rows], d["weight"], d["bias"], sp.topk,
                                         sp.renormalize, sp.num_expert_group, sp.topk_group,
@@ -205,7 +213,7 @@ def time_oracle(name: str, M: int, seconds: float) -> dict:
     the fused workload) repeated until `seconds` of single-thread CPU work."""
     from moe_expert_routing_token_b200 import inputs
     d = inputs.make(name, M)
-    rows = M if name != "fused" else min(M, 4)
+    rows = M if name not in ("fused", "top1") else min(M, 4 if name == "fused" else 256)
     oracle_call(name, d, slice(0, min(rows, 8)))  # compile / warm
     n = 0
     t0 = time.perf_counter()
@@ -324,7 +332,7 @@ def run_ours(args):
     # ---- rotating device pool larger than L2 --------------------------------
     per_set = algorithmic_bytes(name, M)
     pool = max(2, min(256, -(-4 * L2_BYTES // per_set)))
-    if name == "fused":
+    if name in ("fused", "top1"):
         src_x = d["hidden"].to(dev)
         wgt = d["weight"].to(dev)
     else:
@@ -348,6 +356,9 @@ def run_ours(args):
                                            sp.routed_scaling_factor, ws[j].data_ptr(),
                                            ids[j].data_ptr(), None,
                                            wsp[j].data_ptr() if wsp_bytes else None, wsp_bytes, sptr)
+        elif name == "top1":
+            st = lib.moe_fused_router_top1(xs[j].data_ptr(), wgt.data_ptr(), routing.MOE_WEIGHT_E_BY_K, M, sp.K,
+                                           sp.E, sp.softcap, ws[j].data_ptr(), ids[j].data_ptr(), None, sptr)
         elif name in ("softmax", "grouped"):
             st = lib.moe_grouped_topk(xs[j].data_ptr(), dcode, M, sp.E, sp.topk, int(sp.renormalize),
                                       sp.num_expert_group, sp.topk_group, sp.routed_scaling_factor,
@@ -467,9 +478,9 @@ def e2e_measure(name, M, sp, d, dev, stream, world, args):
     from moe_expert_routing_token_b200 import routing
     lib = routing.lib()
     steps = max(1, min(args.steps, 200))
-    src = (d["hidden"] if name == "fused" else d["logits"]).pin_memory()
+    src = (d["hidden"] if name in ("fused", "top1") else d["logits"]).pin_memory()
     x = torch.empty_like(src, device=dev)
-    wgt = d["weight"].to(dev) if name == "fused" else None
+    wgt = d["weight"].to(dev) if name in ("fused", "top1") else None
     bias = d["bias"].to(dev) if d["bias"] is not None else None
     w = torch.empty(M, sp.topk, dtype=torch.float32, device=dev)
     ids = torch.empty(M, sp.topk, dtype=torch.int32, device=dev)
@@ -484,6 +495,8 @@ def e2e_measure(name, M, sp, d, dev, stream, world, args):
             routing.fused_router_topk(x, wgt, bias, sp.topk, sp.renormalize, sp.num_expert_group,
                                       sp.topk_group, sp.routed_scaling_factor, workspace=wsp,
                                       out=(w, ids))
+        elif name == "top1":
+            routing.fused_router_top1(x, wgt, sp.softcap, weight_layout="ek", out=(w, ids))
         elif name in ("softmax", "grouped"):
             routing.grouped_topk(x, sp.topk, sp.renormalize, sp.num_expert_group, sp.topk_group,
                                  sp.routed_scaling_factor, out=(w, ids))

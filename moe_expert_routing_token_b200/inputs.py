@@ -20,6 +20,9 @@ grouped    softmax grouped top-k (DeepSeek-V2 shape): E=160 in 8 groups of 20,
            topk_group=3, k=6, no renormalise, fp32 logits N(0, 1.5^2)
 fused      router projection: hidden bf16 (M, 7168) N(0, 1), router weight bf16
            (7168, 256) N(0, 0.02^2), then the ``biased`` routing
+top1       small-E router projection: hidden bf16 (M, 7168) N(0, 1), router
+           weight bf16 (8, 7168) N(0, 0.02^2) in the (E, K) layout, softcap 30
+           (the pages give no value), then top-1
 =========  =====================================================================
 """
 from __future__ import annotations
@@ -28,7 +31,7 @@ import dataclasses
 
 import torch
 
-WORKLOADS = ("softmax", "sigmoid", "biased", "grouped", "fused")
+WORKLOADS = ("softmax", "sigmoid", "biased", "grouped", "fused", "top1")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -43,8 +46,9 @@ class Workload:
     dtype: torch.dtype          # logits dtype (fused: hidden/weight dtype)
     logit_std: float
     bias_std: float | None      # None: no correction_bias
-    K: int = 0                  # hidden size (fused only)
-    weight_std: float = 0.0     # router weight std (fused only)
+    K: int = 0                  # hidden size (fused, top1)
+    weight_std: float = 0.0     # router weight std (fused, top1)
+    softcap: float = 0.0        # logit softcapping constant (top1)
 
 
 SPECS = {
@@ -54,6 +58,8 @@ SPECS = {
     "grouped": Workload("grouped", 160, 6, False, 8, 3, 1.0, torch.float32, 1.5, None),
     "fused": Workload("fused", 256, 8, True, 8, 4, 2.5, torch.bfloat16, 1.0, 0.05,
                       K=7168, weight_std=0.02),
+    "top1": Workload("top1", 8, 1, False, 1, 1, 1.0, torch.bfloat16, 1.0, None,
+                     K=7168, weight_std=0.02, softcap=30.0),
 }
 
 # Token counts the pages' workloads are quoted at.
@@ -63,6 +69,7 @@ SIZES = {
     "biased": (4096, 32),
     "grouped": (16384,),
     "fused": (8192, 64),
+    "top1": (8192, 64),
 }
 
 
@@ -78,9 +85,9 @@ def _normal(gen: torch.Generator, shape, std: float, dtype: torch.dtype) -> torc
 def make(name: str, M: int, seed: int | None = None) -> dict:
     """Return a dict of CPU tensors for workload ``name`` with ``M`` tokens.
 
-    Keys: ``logits`` (M, E) [not for fused], ``bias`` (E,) fp32 or None,
-    ``hidden`` (M, K) and ``weight`` (K, E) [fused only], plus ``spec`` and
-    ``seed``.
+    Keys: ``logits`` (M, E) [not for fused or top1], ``bias`` (E,) fp32 or
+    None, ``hidden`` (M, K) and ``weight`` [fused: (K, E); top1: (E, K)], plus
+    ``spec`` and ``seed``.
     """
     spec = SPECS[name]
     seed = default_seed(name, M) if seed is None else int(seed)
@@ -89,6 +96,9 @@ def make(name: str, M: int, seed: int | None = None) -> dict:
     if name == "fused":
         out["hidden"] = _normal(gen, (M, spec.K), spec.logit_std, spec.dtype)
         out["weight"] = _normal(gen, (spec.K, spec.E), spec.weight_std, spec.dtype)
+    elif name == "top1":
+        out["hidden"] = _normal(gen, (M, spec.K), spec.logit_std, spec.dtype)
+        out["weight"] = _normal(gen, (spec.E, spec.K), spec.weight_std, spec.dtype)
     else:
         out["logits"] = _normal(gen, (M, spec.E), spec.logit_std, spec.dtype)
     out["bias"] = (None if spec.bias_std is None

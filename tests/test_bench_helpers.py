@@ -33,3 +33,19 @@ def test_algorithmic_bytes():
     # fused: hidden + weight + outputs + bias
     assert bench.algorithmic_bytes("fused", 8192) == 8192 * 7168 * 2 + 7168 * 256 * 2 + 8192 * 64 + 1024
     assert bench.perm_bytes(16384) == 16384 * 8 * 20 + (2 * 256 + 1) * 4
+
+
+def test_top1_workload():
+    from moe_expert_routing_token_b200 import inputs
+    # hidden + the (E, K) weight + one (weight, id) pair per token; no bias
+    assert bench.algorithmic_bytes("top1", 8192) == 8192 * 7168 * 2 + 8 * 7168 * 2 + 8192 * 8
+    d = bench.workload_desc("top1", 64)
+    assert d["K"] == 7168 and d["softcap"] == 30.0 and d["E"] == 8 and d["topk"] == 1
+    x = inputs.make("top1", 6)
+    assert tuple(x["hidden"].shape) == (6, 7168) and tuple(x["weight"].shape) == (8, 7168)
+    assert x["bias"] is None and "logits" not in x
+    r, _ = bench.oracle_call("top1", x, slice(0, 6))
+    assert r.ids.shape == (6, 1) and (r.weights > 0).all() and (r.weights <= 1).all()
+    # the new workload leaves the other workloads' seeds (and so their draws) as they were
+    assert [inputs.default_seed(n, 16384) for n in ("softmax", "sigmoid", "biased", "grouped", "fused")] == \
+        [1015, 2015, 3015, 4015, 5015]

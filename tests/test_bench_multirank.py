@@ -35,7 +35,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_ranks_max_time_and_sharded_rows():
     world = 2
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:  # no fork of a threaded test process
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
