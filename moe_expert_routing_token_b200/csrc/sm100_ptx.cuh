@@ -230,9 +230,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
-// this CTA's shared memory to shared memory of a CTA in the cluster (no
-// multicast); completes `bytes` of transaction count on the mbarrier at
-// `mbar_cluster` in the destination CTA.
+// this CTA's shared memory to shared memory of one other CTA in the cluster
+// (a single destination); completes `bytes` of transaction count on the
+// mbarrier at `mbar_cluster` in the destination CTA.
 __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
                                                      uint32_t mbar_cluster) {
     asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
