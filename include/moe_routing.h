@@ -292,7 +292,7 @@ MOE_API int moe_fused_router_topk_noalloc(const void* hidden_states, const void*
  *   topk_ids        device, (M, 1) int32 out
  *   logits_out      device, (M, E) fp32 out, or NULL (debug: the raw logits)
  * Every batch size runs on the CUDA cores: at E <= 8 the projection does at
- * most 8 flops per byte of hidden state, so it streams at HBM bandwidth (the
+ * most 8 flops per byte of hidden state, below the fp32 CUDA-core ridge (the
  * page's batch-size switch to tensor cores has no counterpart here).
  * Asynchronous on `stream`; no allocation; M == 0 launches nothing.
  */

@@ -12,9 +12,10 @@
 // distinct logits into one capped value.
 //
 // With E <= 8 experts the work is 2 * E flops per 2-byte hidden value, below
-// the B200's fp32 ridge, so the kernel streams the hidden states at HBM
-// bandwidth on the CUDA cores at every batch size; the tensor cores would
-// only add a second pass over the accumulator.  Each 128-thread block takes
+// the B200's fp32 CUDA-core ridge (about 11 flops per byte), so one kernel
+// serves every batch size.  At E = 8 the instruction issue (the FMAs plus the
+// bf16 unpacking) is close to the rate at which HBM delivers the hidden
+// states, so E = 8 sits near the balance of the two.  Each 128-thread block takes
 // 4 rows at a time; every thread walks 8-value chunks of the hidden size,
 // loads the chunk's weights once (E 16-byte vectors, cached in L1/L2) and
 // applies them to the 4 rows.  The partial sums meet through warp shuffles
