@@ -50,6 +50,15 @@ MUTANTS = {
     "softcap_unscaled": ("out[i] = c * tanh(x[i] / c);", "out[i] = tanh(x[i] / c);"),
     "softcap_times_inside": ("out[i] = c * tanh(x[i] / c);", "out[i] = c * tanh(x[i] * c);"),
     "softcap_zero_clears": ("            out[i] = x[i];\n", "            out[i] = 0.0;\n"),
+    "router_skips_last_term": ("for (int c = 0; c < K; ++c) {", "for (int c = 0; c < K - 1; ++c) {"),
+    "gate_by_sorted_position": ("if (weights && gate) gate[p] = weights[i];",
+                                "if (weights && gate) gate[p] = weights[p];"),
+    "top2_second_skips_first_slot": ("if (j != best_j && s[first + j] > second) second = s[first + j];",
+                                     "if (s[first + j] > second && j != 0) second = s[first + j];"),
+    "renorm_epsilon": ("if (renorm) w = w / wsum;", "if (renorm) w = w / (wsum + 1e-9);"),
+    "shared_sum_includes_own_slot": ("for (int j = 0; j < k - 1; ++j) sum += weights[i * (int64_t)k + j];",
+                                     "for (int j = 0; j < k; ++j) sum += weights[i * (int64_t)k + j];"),
+    "sigmoid_half_slope": ("p[e] = 1.0 / (1.0 + exp(-x[e]));", "p[e] = 1.0 / (1.0 + exp(-0.5 * x[e]));"),
 }
 
 
