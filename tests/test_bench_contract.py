@@ -12,7 +12,7 @@ KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_
         "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
 
 
-@pytest.mark.parametrize("workload", ["sigmoid", "permute"])
+@pytest.mark.parametrize("workload", ["sigmoid", "permute", "top1"])
 def test_reference_arm_record(workload):
     res = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", workload,
                           "--steps", "2", "--warmup", "1", "--cpu-seconds", "0.5"],

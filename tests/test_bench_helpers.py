@@ -49,3 +49,11 @@ def test_top1_workload():
     # the new workload leaves the other workloads' seeds (and so their draws) as they were
     assert [inputs.default_seed(n, 16384) for n in ("softmax", "sigmoid", "biased", "grouped", "fused")] == \
         [1015, 2015, 3015, 4015, 5015]
+
+
+def test_metric_labels():
+    # the default workload keeps the headline metric's exact text
+    assert bench.metric_for("sigmoid") == bench.METRIC == \
+        "routed tokens/s & µs/call (E=256,k=8 biased grouped top-k); % of HBM roofline"
+    assert bench.metric_for("biased") == bench.METRIC
+    assert "E=8" in bench.metric_for("top1") and "tensor" in bench.metric_for("fused")
