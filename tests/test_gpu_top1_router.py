@@ -17,6 +17,7 @@ import torch
 
 import moe_expert_routing_token_b200 as moe
 import oracle
+from moe_expert_routing_token_b200 import inputs
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -89,6 +90,15 @@ def _check(h, w_ek, layout, c):
 def test_top1_router(M, K, E, layout, c):
     h, w = _draw(M, K, E, seed=M + K + E)
     _check(h, w, layout, c)
+
+
+def test_bench_workload_full_size():
+    """The configuration bench.py times: the seeded top1 workload, M = 8192,
+    hidden 7168, the (E, K) weight, softcap 30; every row against the oracle."""
+    d = inputs.make("top1", 8192)
+    sp = d["spec"]
+    rep = _check(d["hidden"], d["weight"], "ek", sp.softcap)
+    assert rep.near_tie <= 8192 // 200, rep.summary()
 
 
 @pytest.mark.parametrize("E", [5, 6, 7])
