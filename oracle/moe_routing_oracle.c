@@ -291,7 +291,12 @@ int oracle_softcap(const double* x, int64_t n, double c, double* out) {
  *   scatter[i]     the sorted position of pair i (gather[scatter[i]] == i)
  *   gate[p]        weights[gather[p]] (NULL weights or gate: skipped)
  * A pair whose id lies outside [0, E) is skipped: not counted, not placed,
- * scatter = -1 (offsets[E] is then the number of placed pairs).
+ * scatter = -1 (offsets[E] is then the number of placed pairs).  Reason: the
+ * routing page's shared-expert slot (§6, 공유 전문가 슬롯 할당) writes ids
+ * E .. E + n_shared - 1 into topk_ids, so a routing result handed to a
+ * permutation over the E routed experts can carry ids that name no expert of
+ * that sort; those pairs get no position.  A negative id (a pair masked out
+ * before this step) is read the same way.
  * ------------------------------------------------------------------------- */
 int oracle_expert_permutation(const int32_t* ids, const double* weights, int64_t M, int k, int E,
                               int32_t* counts, int32_t* offsets, int32_t* gather, int32_t* scatter,

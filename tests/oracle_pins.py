@@ -224,15 +224,44 @@ def check_library(lib, seed=5) -> list[str]:
 
 
 def check_permutation_golden(lib) -> list[str]:
-    doc = json.load(open(os.path.join(GOLDEN, "expert_permutation_small.json")))
-    p = oracle.expert_permutation(np.asarray(doc["topk_ids"], np.int32), doc["num_experts"],
-                                  np.asarray(doc["topk_weights"], np.float64), lib=lib)
+    """Hand-worked cases: a plain one, and one whose ids include a shared-expert
+    slot (id E, the routing page's §6) and a masked pair (id -1).  Only the
+    first offsets[E] entries of gather and gate are defined."""
     fails = []
-    for key in ("counts", "offsets", "gather", "scatter"):
-        if getattr(p, key).tolist() != doc[key]:
-            fails.append(f"permutation hand case: {key} {getattr(p, key).tolist()} != {doc[key]}")
-    if p.gate.tolist() != doc["gate"]:
-        fails.append(f"permutation hand case: gate {p.gate.tolist()}")
+    for name in ("expert_permutation_small.json", "expert_permutation_out_of_range.json"):
+        doc = json.load(open(os.path.join(GOLDEN, name)))
+        p = oracle.expert_permutation(np.asarray(doc["topk_ids"], np.int32), doc["num_experts"],
+                                      np.asarray(doc["topk_weights"], np.float64), lib=lib)
+        placed = int(p.offsets[-1])
+        got = {"counts": p.counts.tolist(), "offsets": p.offsets.tolist(), "gather": p.gather[:placed].tolist(),
+               "scatter": p.scatter.tolist(), "gate": p.gate[:placed].tolist()}
+        for key, val in got.items():
+            if val != doc[key]:
+                fails.append(f"permutation hand case {name}: {key} {val} != {doc[key]}")
+    return fails
+
+
+def check_permutation_after_shared_slot(lib, seed=29) -> list[str]:
+    """The routing page's §6 writes the shared expert's id E + j into the last
+    slot; a permutation over the E routed experts then places exactly the
+    other k - 1 slots of every row, in the order it gives them without the
+    shared slot (pair indices mapped from (token, slot) over k - 1 to k)."""
+    rng = np.random.default_rng(seed)
+    fails = []
+    M, k, E, n_shared = 50, 4, 12, 2
+    x = rng.normal(0, 2, size=(M, E))
+    r = oracle.topk_softmax(x, k, True, lib=lib)
+    w_sh, ids_sh = oracle.fill_shared_slot(r.weights, r.ids, E, n_shared, rng.integers(0, n_shared, M), 2.0,
+                                           lib=lib)
+    full = oracle.expert_permutation(ids_sh, E, w_sh, lib=lib)
+    part = oracle.expert_permutation(ids_sh[:, : k - 1], E, w_sh[:, : k - 1], lib=lib)
+    to_full = (part.gather[: int(part.offsets[-1])] // (k - 1)) * k + part.gather[: int(part.offsets[-1])] % (k - 1)
+    if not np.array_equal(full.counts, part.counts) or not np.array_equal(full.offsets, part.offsets):
+        fails.append("shared slot: counts or offsets include the shared expert's pairs")
+    if not np.array_equal(full.gather[: int(full.offsets[-1])], to_full):
+        fails.append("shared slot: placed pairs differ from the permutation without that slot")
+    if not np.all(full.scatter.reshape(M, k)[:, k - 1] == -1):
+        fails.append("shared slot: a shared-expert pair has a position")
     return fails
 
 
@@ -363,7 +392,8 @@ def check_fused_top1(lib) -> list[str]:
 
 
 ALL_CHECKS = (check_golden, check_router_golden, check_router_numpy, check_brute, check_library,
-              check_permutation_golden, check_permutation_numpy, check_postprocess, check_softcap,
+              check_permutation_golden, check_permutation_after_shared_slot, check_permutation_numpy,
+              check_postprocess, check_softcap,
               check_fused_top1)
 
 

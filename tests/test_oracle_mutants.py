@@ -58,6 +58,8 @@ MUTANTS = {
     "renorm_epsilon": ("if (renorm) w = w / wsum;", "if (renorm) w = w / (wsum + 1e-9);"),
     "shared_sum_includes_own_slot": ("for (int j = 0; j < k - 1; ++j) sum += weights[i * (int64_t)k + j];",
                                      "for (int j = 0; j < k; ++j) sum += weights[i * (int64_t)k + j];"),
+    "perm_counts_high_ids": ("        if (ids[i] >= 0 && ids[i] < E) counts[ids[i]] += 1;",
+                             "        if (ids[i] >= 0 && ids[i] <= E) counts[ids[i] < E ? ids[i] : E - 1] += 1;"),
     "sigmoid_half_slope": ("p[e] = 1.0 / (1.0 + exp(-x[e]));", "p[e] = 1.0 / (1.0 + exp(-0.5 * x[e]));"),
 }
 
