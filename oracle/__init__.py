@@ -22,6 +22,8 @@ Operations (each a restatement of the SGLang MoE routing page,
 * :func:`softcap_logits`      - §5 softcapping, c * tanh(logits / c)
 * :func:`fused_router_top1`   - §5 projection, softcapping and softmax top-1
   (weight = 1 / sum_e exp(l_e - max l), the page's invsumexp)
+* :func:`philox4x64`, :func:`shared_pick_philox` - the §6 shared-expert draw
+  from a seed (Philox4x64-10 of Salmon et al., SC'11)
 """
 from __future__ import annotations
 
@@ -43,6 +45,7 @@ GROUP_MAX, GROUP_TOP2_SUM = 0, 1
 
 _DBL = ctypes.POINTER(ctypes.c_double)
 _I32 = ctypes.POINTER(ctypes.c_int32)
+_U64 = ctypes.POINTER(ctypes.c_uint64)
 
 
 def compile_oracle(src: str = _SRC, out: str = _LIB_PATH) -> str:
@@ -72,6 +75,10 @@ def _bind(path: str):
     lib.oracle_fill_shared_slot.restype = ctypes.c_int
     lib.oracle_fill_shared_slot.argtypes = [_DBL, _I32, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             _I32, ctypes.c_double]
+    lib.oracle_philox4x64.restype = None
+    lib.oracle_philox4x64.argtypes = [_U64, _U64, _U64]
+    lib.oracle_shared_pick_philox.restype = ctypes.c_int
+    lib.oracle_shared_pick_philox.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64, _I32]
     lib.oracle_sort_by_id.restype = ctypes.c_int
     lib.oracle_sort_by_id.argtypes = [_DBL, _I32, ctypes.c_int64, ctypes.c_int]
     lib.oracle_expert_permutation.restype = ctypes.c_int
@@ -251,6 +258,29 @@ def expert_permutation(topk_ids, num_experts: int, topk_weights=None, lib=None) 
     if rc != 0:
         raise ValueError("oracle_expert_permutation: invalid arguments")
     return Permutation(counts, offsets, gather, scatter, gate)
+
+
+def philox4x64(counter, key, lib=None) -> np.ndarray:
+    """Philox4x64-10 (oracle_philox4x64): four uint64 outputs of one block for
+    a counter of four words and a key of two."""
+    c = np.ascontiguousarray(np.asarray(counter, dtype=np.uint64))
+    k = np.ascontiguousarray(np.asarray(key, dtype=np.uint64))
+    if c.shape != (4,) or k.shape != (2,):
+        raise ValueError("counter has 4 words, key has 2")
+    out = np.zeros(4, np.uint64)
+    (lib or load()).oracle_philox4x64(_ptr(c, _U64), _ptr(k, _U64), _ptr(out, _U64))
+    return out
+
+
+def shared_pick_philox(M: int, num_shared: int, seed: int, offset: int = 0, lib=None) -> np.ndarray:
+    """The seeded shared-expert draw (oracle_shared_pick_philox): int32 (M,)
+    values in [0, num_shared)."""
+    pick = np.zeros(max(0, int(M)), np.int32)
+    rc = (lib or load()).oracle_shared_pick_philox(int(M), int(num_shared), int(seed) & (2**64 - 1),
+                                                  int(offset) & (2**64 - 1), _ptr(pick, _I32))
+    if rc != 0:
+        raise ValueError("oracle_shared_pick_philox: invalid arguments")
+    return pick
 
 
 def fill_shared_slot(topk_weights, topk_ids, num_experts: int, num_shared: int, picks,

@@ -349,6 +349,62 @@ int oracle_fill_shared_slot(double* weights, int32_t* ids, int64_t M, int k, int
 }
 
 /* ---------------------------------------------------------------------------
+ * oracle_philox4x64: the Philox4x64-10 counter-based generator of Salmon,
+ * Moraes, Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3"
+ * (SC'11).  Ten rounds on a counter of four 64-bit words under a key of two;
+ * a round multiplies words 0 and 2 by the two Philox constants and forms
+ *   (hi(M1 x2) ^ x1 ^ k0,  lo(M1 x2),  hi(M0 x0) ^ x3 ^ k1,  lo(M0 x0)),
+ * and the key is bumped by the two Weyl constants before every round but the
+ * first.  out may not alias ctr.
+ * ------------------------------------------------------------------------- */
+void oracle_philox4x64(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4]) {
+    const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+    uint64_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint64_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += W0;
+            k1 += W1;
+        }
+        const unsigned __int128 p0 = (unsigned __int128)M0 * x0;
+        const unsigned __int128 p1 = (unsigned __int128)M1 * x2;
+        const uint64_t hi0 = (uint64_t)(p0 >> 64), lo0 = (uint64_t)p0;
+        const uint64_t hi1 = (uint64_t)(p1 >> 64), lo1 = (uint64_t)p1;
+        const uint64_t y0 = hi1 ^ x1 ^ k0, y1 = lo1, y2 = hi0 ^ x3 ^ k1, y3 = lo0;
+        x0 = y0;
+        x1 = y1;
+        x2 = y2;
+        x3 = y3;
+    }
+    out[0] = x0;
+    out[1] = x1;
+    out[2] = x2;
+    out[3] = x3;
+}
+
+/* ---------------------------------------------------------------------------
+ * oracle_shared_pick_philox: the random shared-expert draw of [R] §6
+ * (torch.randint(num_experts, num_experts + num_fused_shared_experts), one
+ * per token) made reproducible from a seed.  The pages name no generator;
+ * the reading taken: token i draws u = word 0 of Philox4x64-10 with counter
+ * (offset + i as a 128-bit number in words 0-1, 0, 0) and key (seed, 0), and
+ * picks floor(u * num_shared / 2^64), the high word of the 128-bit product.
+ * ------------------------------------------------------------------------- */
+int oracle_shared_pick_philox(int64_t M, int num_shared, uint64_t seed, uint64_t offset, int32_t* pick) {
+    if (M < 0 || num_shared < 1) return ORACLE_BAD_ARGS;
+    const uint64_t key[2] = {seed, 0};
+    for (int64_t i = 0; i < M; ++i) {
+        const uint64_t c0 = offset + (uint64_t)i;
+        const uint64_t ctr[4] = {c0, c0 < offset ? 1u : 0u, 0, 0};
+        uint64_t out[4];
+        oracle_philox4x64(ctr, key, out);
+        pick[i] = (int32_t)(uint64_t)(((unsigned __int128)out[0] * (uint64_t)num_shared) >> 64);
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
  * oracle_sort_by_id: reorder every row's k (weight, id) pairs by ascending
  * id, equal ids keeping their order - the ascending expert/block-id output
  * that [M] 코드 분석 §1 (minimax_decode_topk) produces with a warp rank sort.

@@ -391,9 +391,45 @@ def check_fused_top1(lib) -> list[str]:
     return fails
 
 
+def check_philox(lib) -> list[str]:
+    """The seeded shared-expert draw: Philox4x64-10 against numpy's
+    implementation of the same generator (numpy advances its counter once
+    before the first block, so numpy at counter c gives the block at c + 1),
+    the pick mapping floor(u n / 2^64) against its closed form for n = 2^j
+    (the top j bits of u), the counter carry past 2^64, and the range."""
+    fails = []
+    for c0, k0, k1 in [(0, 0, 0), (41, 123456789, 987654321), (2**40 + 3, 2**63 + 5, 17)]:
+        got = oracle.philox4x64([c0 + 1, 0, 0, 0], [k0, k1], lib=lib)
+        ref = np.random.Philox(counter=np.array([c0, 0, 0, 0], np.uint64),
+                               key=np.array([k0, k1], np.uint64)).random_raw(4)
+        if not np.array_equal(got, ref.astype(np.uint64)):
+            fails.append(f"philox4x64 counter {c0 + 1} key ({k0}, {k1}) differs from numpy's Philox")
+    # the draw is word 0 of the block at counter offset + i, key (seed, 0)
+    seed, offset, M = 20250, 7, 64
+    raw = np.array([oracle.philox4x64([offset + i, 0, 0, 0], [seed, 0], lib=lib)[0] for i in range(M)],
+                   dtype=np.uint64)
+    for j in (0, 1, 3, 5):
+        pick = oracle.shared_pick_philox(M, 2 ** j, seed, offset, lib=lib)
+        expect = (raw >> np.uint64(64 - j)).astype(np.int64) if j else np.zeros(M, np.int64)
+        if not np.array_equal(pick.astype(np.int64), expect):
+            fails.append(f"shared pick with n = 2^{j} is not the top {j} bits of the Philox word")
+    # counter carry: offset + i passes 2^64 into word 1
+    top = 2**64 - 2
+    pick = oracle.shared_pick_philox(4, 2**5, seed, top, lib=lib)
+    words = [oracle.philox4x64([(top + i) % 2**64, (top + i) >> 64, 0, 0], [seed, 0], lib=lib)[0] for i in range(4)]
+    if pick.tolist() != [int(w) >> 59 for w in words]:
+        fails.append("shared pick: the counter does not carry into its second word past 2^64")
+    # range and a loose uniformity check for a non-power-of-two count
+    pick = oracle.shared_pick_philox(30000, 3, 99, 0, lib=lib)
+    counts = np.bincount(pick, minlength=3)
+    if pick.min() < 0 or pick.max() > 2 or np.any(np.abs(counts - 10000) > 600):
+        fails.append(f"shared pick over 3 values: counts {counts.tolist()}")
+    return fails
+
+
 ALL_CHECKS = (check_golden, check_router_golden, check_router_numpy, check_brute, check_library,
               check_permutation_golden, check_permutation_after_shared_slot, check_permutation_numpy,
-              check_postprocess, check_softcap,
+              check_postprocess, check_philox, check_softcap,
               check_fused_top1)
 
 

@@ -60,6 +60,13 @@ MUTANTS = {
                                      "for (int j = 0; j < k; ++j) sum += weights[i * (int64_t)k + j];"),
     "perm_counts_high_ids": ("        if (ids[i] >= 0 && ids[i] < E) counts[ids[i]] += 1;",
                              "        if (ids[i] >= 0 && ids[i] <= E) counts[ids[i] < E ? ids[i] : E - 1] += 1;"),
+    "philox_no_key_bump": ("            k0 += W0;\n", "            k0 += 0;\n"),
+    "philox_words_swapped": ("y0 = hi1 ^ x1 ^ k0, y1 = lo1, y2 = hi0 ^ x3 ^ k1, y3 = lo0;",
+                             "y0 = hi0 ^ x1 ^ k0, y1 = lo0, y2 = hi1 ^ x3 ^ k1, y3 = lo1;"),
+    "pick_low_bits": ("pick[i] = (int32_t)(uint64_t)(((unsigned __int128)out[0] * (uint64_t)num_shared) >> 64);",
+                      "pick[i] = (int32_t)(out[0] % (uint64_t)num_shared);"),
+    "pick_no_carry": ("const uint64_t ctr[4] = {c0, c0 < offset ? 1u : 0u, 0, 0};",
+                      "const uint64_t ctr[4] = {c0, 0, 0, 0};"),
     "sigmoid_half_slope": ("p[e] = 1.0 / (1.0 + exp(-x[e]));", "p[e] = 1.0 / (1.0 + exp(-0.5 * x[e]));"),
 }
 
