@@ -59,8 +59,10 @@ extern "C" {
  * fused router, the softcap and aiter variants, the expert permutation, the
  * shared-expert slot, the ascending-id order and the bounded-wait self-test
  * (every version-1 call keeps its signature and meaning).  3: adds the
- * small-E top-1 router moe_fused_router_top1 (earlier calls unchanged). */
-#define MOE_ROUTING_ABI_VERSION 3
+ * small-E top-1 router moe_fused_router_top1 (earlier calls unchanged).  4:
+ * adds moe_fill_shared_expert_slot_philox, the shared-expert slot with the
+ * library drawing the shared expert from a seed (earlier calls unchanged). */
+#define MOE_ROUTING_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -348,6 +350,25 @@ MOE_API int moe_expert_permutation(const int32_t* topk_ids, const float* topk_we
 MOE_API int moe_fill_shared_expert_slot(float* topk_weights, int32_t* topk_ids, int64_t M, int32_t k, int32_t E,
                                         int32_t num_shared, const int32_t* shared_pick,
                                         float routed_scaling_factor, void* stream);
+
+/*
+ * moe_fill_shared_expert_slot_philox - moe_fill_shared_expert_slot with the
+ * random draw made by the library from a seed, so that a caller needs no
+ * device-side random numbers of its own.  The routing page (§6) draws
+ * torch.randint(E, E + num_shared) per token and names no generator; this
+ * call uses Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random
+ * numbers: as easy as 1, 2, 3", SC'11), a counter-based generator:
+ *     u_i    = word 0 of Philox4x64-10(counter = (offset + i, carry, 0, 0),
+ *                                      key = (seed, 0))
+ *     pick_i = floor(u_i * num_shared / 2^64)         (in [0, num_shared))
+ * for row i, the counter being offset + i as a 128-bit number.  The same
+ * (seed, offset) always gives the same picks; advance offset by M between
+ * calls for fresh draws.  Other arguments and the weight rule are those of
+ * moe_fill_shared_expert_slot.  k <= 32; M = 0 is a no-op.
+ */
+MOE_API int moe_fill_shared_expert_slot_philox(float* topk_weights, int32_t* topk_ids, int64_t M, int32_t k,
+                                               int32_t E, int32_t num_shared, uint64_t seed, uint64_t offset,
+                                               float routed_scaling_factor, void* stream);
 
 /*
  * moe_sort_topk_by_id - reorder every row's k (weight, id) pairs by ascending

@@ -14,6 +14,7 @@ from .routing import (  # noqa: F401
     expert_permutation,
     expert_permutation_workspace_size,
     fill_shared_expert_slot,
+    fill_shared_expert_slot_philox,
     fused_router_top1,
     fused_router_topk,
     fused_router_workspace_size,
@@ -27,5 +28,5 @@ from .routing import (  # noqa: F401
 __all__ = [
     "topk_softmax", "grouped_topk", "biased_grouped_topk", "fused_router_topk",
     "fused_router_workspace_size", "lib", "RoutingError", "watchdog_trips", "expert_permutation",
-    "expert_permutation_workspace_size", "fill_shared_expert_slot", "sort_topk_by_id", "fused_router_top1",
+    "expert_permutation_workspace_size", "fill_shared_expert_slot", "fill_shared_expert_slot_philox", "sort_topk_by_id", "fused_router_top1",
 ]

@@ -54,6 +54,8 @@ SIGNATURES = {
                                              _vp]),
     "moe_expert_permutation_workspace_size": (_sz, [_i64, _i32, _i32]),
     "moe_fill_shared_expert_slot": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _i32, _vp, _f32, _vp]),
+    "moe_fill_shared_expert_slot_philox": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _i32, ctypes.c_uint64,
+                                                           ctypes.c_uint64, _f32, _vp]),
     "moe_sort_topk_by_id": (ctypes.c_int, [_vp, _vp, _i64, _i32, _vp]),
     "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, _vp, _vp]),
     "moe_expert_permutation": (ctypes.c_int, [_vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
@@ -362,6 +364,22 @@ def fill_shared_expert_slot(topk_weights: torch.Tensor, topk_ids: torch.Tensor, 
                                                int(num_experts), int(num_shared), shared_pick.data_ptr(), rsf,
                                                _stream(topk_ids.device))
     _check(st, "moe_fill_shared_expert_slot")
+    return topk_weights, topk_ids
+
+
+def fill_shared_expert_slot_philox(topk_weights: torch.Tensor, topk_ids: torch.Tensor, num_experts: int,
+                                   num_shared: int, seed: int, offset: int = 0, routed_scaling_factor=None):
+    """As fill_shared_expert_slot, with the shared expert of row i drawn by
+    the library: Philox4x64-10 at counter offset + i under key (seed, 0)."""
+    M, k = _result_pair(topk_weights, topk_ids)
+    rsf = 0.0 if routed_scaling_factor is None else float(routed_scaling_factor)
+    if routed_scaling_factor is not None and rsf == 0.0:
+        raise ValueError("routed_scaling_factor 0 is reserved for None")
+    with _on(topk_ids.device):
+        st = lib().moe_fill_shared_expert_slot_philox(topk_weights.data_ptr(), topk_ids.data_ptr(), M, k,
+                                                      int(num_experts), int(num_shared), int(seed) & (2**64 - 1),
+                                                      int(offset) & (2**64 - 1), rsf, _stream(topk_ids.device))
+    _check(st, "moe_fill_shared_expert_slot_philox")
     return topk_weights, topk_ids
 
 

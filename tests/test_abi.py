@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 3
+    assert lib.moe_abi_version() == 4
     assert lib.moe_status_string(0) == b"MOE_OK"
     assert lib.moe_status_string(1) == b"MOE_ERR_INVALID_ARG"
     assert lib.moe_status_string(2) == b"MOE_ERR_UNSUPPORTED"
@@ -153,6 +153,13 @@ def test_postprocess_validation(lib):
     assert lib.moe_fill_shared_expert_slot(P, P, 4, 9, 256, 1, None, 2.5, None) == 1    # no picks
     assert lib.moe_fill_shared_expert_slot(P, P, 4, 9, 256, 1, P, float("nan"), None) == 1
     assert lib.moe_fill_shared_expert_slot(P, P, 0, 9, 256, 1, None, 2.5, None) == 0    # empty: no launch
+    # (weights, ids, M, k, E, num_shared, seed, offset, rsf, stream)
+    assert lib.moe_fill_shared_expert_slot_philox(P, P, 4, 0, 256, 1, 7, 0, 2.5, None) == 1     # k < 1
+    assert lib.moe_fill_shared_expert_slot_philox(P, P, 4, 33, 256, 1, 7, 0, 2.5, None) == 2    # k > 32
+    assert lib.moe_fill_shared_expert_slot_philox(P, P, 4, 9, 256, 0, 7, 0, 2.5, None) == 1     # no shared expert
+    assert lib.moe_fill_shared_expert_slot_philox(P, P, 4, 9, 256, 1, 7, 0, float("nan"), None) == 1
+    assert lib.moe_fill_shared_expert_slot_philox(None, P, 4, 9, 256, 1, 7, 0, 2.5, None) == 1  # null weights
+    assert lib.moe_fill_shared_expert_slot_philox(P, P, 0, 9, 256, 1, 7, 0, 2.5, None) == 0     # empty: no launch
     assert lib.moe_sort_topk_by_id(P, None, 4, 8, None) == 1
     assert lib.moe_sort_topk_by_id(P, P, 4, 40, None) == 2
     assert lib.moe_sort_topk_by_id(P, P, 0, 8, None) == 0

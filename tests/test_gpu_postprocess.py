@@ -67,3 +67,49 @@ def test_fill_then_sort_composes():
     torch.cuda.synchronize()
     ids_h = ids.cpu().numpy()
     assert np.all(np.diff(ids_h, axis=1) >= 0) and np.all(ids_h[:, -1] == 256)
+
+
+@pytest.mark.parametrize("M,k,num_shared,seed,offset", [
+    (1, 9, 1, 0, 0),
+    (1000, 9, 3, 2025, 0),
+    (16384, 9, 2, 7, 123456789),
+    (4097, 9, 5, 2**63 + 11, 2**64 - 100),   # the counter carries into its second word
+    (257, 32, 7, 99, 5),
+])
+@pytest.mark.parametrize("rsf", [2.5, None])
+def test_fill_shared_expert_slot_philox(M, k, num_shared, seed, offset, rsf):
+    """The library's seeded draw: the shared experts bit-exact with the
+    oracle's Philox4x64-10 picks; the weights as for the explicit draw."""
+    if k == 32:
+        g = torch.Generator().manual_seed(M)
+        w = torch.rand(M, k, generator=g).to(DEV)
+        ids = torch.randint(0, 256, (M, k), generator=g, dtype=torch.int32).to(DEV)
+    else:
+        w, ids = _routed(M, k, seed=M + k)
+    w0, ids0 = w.cpu().numpy(), ids.cpu().numpy()
+    moe.fill_shared_expert_slot_philox(w, ids, 256, num_shared, seed, offset, rsf)
+    torch.cuda.synchronize()
+    pick = oracle.shared_pick_philox(M, num_shared, seed, offset)
+    w_ref, ids_ref = oracle.fill_shared_slot(w0, ids0, 256, num_shared, pick, rsf)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    got = w.cpu().numpy().astype(np.float64)
+    assert np.array_equal(got[:, :-1], w0[:, :-1].astype(np.float64))
+    assert np.allclose(got[:, -1], w_ref[:, -1], rtol=max(k - 1, 1) * 2.0**-24, atol=0.0)
+
+
+def test_philox_draws_advance_with_offset():
+    """Consecutive calls with offset advanced by M give the draws of one call
+    over 2M rows; the same (seed, offset) repeats them."""
+    M = 3000
+    w, ids = _routed(2 * M, 9, seed=1)
+    a_w, a_ids = w[:M].clone(), ids[:M].clone()
+    b_w, b_ids = w[M:].clone(), ids[M:].clone()
+    moe.fill_shared_expert_slot_philox(w, ids, 256, 4, 31, 1000, 2.5)
+    moe.fill_shared_expert_slot_philox(a_w, a_ids, 256, 4, 31, 1000, 2.5)
+    moe.fill_shared_expert_slot_philox(b_w, b_ids, 256, 4, 31, 1000 + M, 2.5)
+    torch.cuda.synchronize()
+    assert torch.equal(ids[:M], a_ids) and torch.equal(ids[M:], b_ids)
+    c_w, c_ids = w[:M].clone(), ids[:M].clone()
+    moe.fill_shared_expert_slot_philox(c_w, c_ids, 256, 4, 31, 1000, 2.5)
+    torch.cuda.synchronize()
+    assert torch.equal(c_ids, a_ids)
