@@ -11,11 +11,13 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <unordered_map>
 
 #include "fused_router.cuh"
 #include "moe_routing.h"
+#include "routing_direct.cuh"
 #include "routing_kernels.cuh"
 #include "routing_staged.cuh"
 #include "routing_stream.cuh"
@@ -43,7 +45,7 @@ int cuda_fail(cudaError_t err, const char* what) {
 struct LaunchCache {
     std::mutex mu;
     std::unordered_map<int, int> sms;
-    std::unordered_map<const void*, int> per_sm[64];
+    std::unordered_map<int, std::unordered_map<const void*, int>> per_sm;  // device -> kernel -> blocks
 };
 LaunchCache& cache() {
     static LaunchCache c;
@@ -73,7 +75,7 @@ int resident_blocks(int dev, Kernel k, int threads, size_t smem, int* out) {
     LaunchCache& c = cache();
     const void* key = reinterpret_cast<const void*>(k);
     std::lock_guard<std::mutex> lk(c.mu);
-    auto& m = c.per_sm[dev & 63];
+    auto& m = c.per_sm[dev];
     auto it = m.find(key);
     if (it != m.end()) {
         *out = it->second;
@@ -144,13 +146,13 @@ int launch_ring(RingKernel kern, size_t smem, int threads, int box_e, int rb, co
     if (rc != MOE_OK) return rc;
     {
         static std::mutex mu;
-        static std::unordered_map<const void*, uint64_t> done;  // kernel -> devices done (bit mask)
+        static std::unordered_map<int, std::unordered_map<const void*, bool>> done;  // device -> kernel -> set
         std::lock_guard<std::mutex> lk(mu);
-        uint64_t& bits = done[reinterpret_cast<const void*>(kern)];
-        if (!(bits & (1ull << (dev & 63)))) {
+        bool& set = done[dev][reinterpret_cast<const void*>(kern)];
+        if (!set) {
             cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (err != cudaSuccess) return cuda_fail(err, what);
-            bits |= 1ull << (dev & 63);
+            set = true;
         }
     }
     rc = resident_blocks(dev, kern, threads, smem, &per_sm);
@@ -234,9 +236,95 @@ int launch_generic(const RouteArgs& a, cudaStream_t st) {
                        warps, a, st);
 }
 
+// Direct kernel: raise its dynamic shared memory limit once per device, size
+// the grid to the octets (R rows per warp) capped at one wave of resident
+// blocks, and launch with programmatic dependent launch (the kernel waits for
+// the previous kernel before it reads any input).
+template <typename TIn, int E, int SCORE, bool BIAS, int MODE, int GS>
+int launch_direct(const RouteArgs& a, cudaStream_t st) {
+    auto kern = route_direct_kernel<TIn, E, SCORE, BIAS, MODE, GS>;
+    constexpr size_t smem = direct_smem_bytes<TIn, E>();
+    int dev = 0, sms = 0, per_sm = 1;
+    int rc = device_and_sms(&dev, &sms);
+    if (rc != MOE_OK) return rc;
+    {
+        static std::mutex mu;
+        static std::unordered_map<int, bool> done;  // device ordinal -> attribute set
+        std::lock_guard<std::mutex> lk(mu);
+        if (!done[dev]) {
+            cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (err != cudaSuccess) return cuda_fail(err, "direct routing kernel attribute");
+            done[dev] = true;
+        }
+    }
+    rc = resident_blocks(dev, kern, kDirectThreads, smem, &per_sm);
+    if (rc != MOE_OK) return rc;
+    using Shape = DirectShape<TIn, E>;
+    constexpr int R = Shape::R;
+    const int64_t n_oct = (a.M + R - 1) / R;
+    // E = 256: the logits seen as rows of 128 bytes, one box of R token rows
+    // per copy, 128-byte swizzle
+    CUtensorMap tmap;
+    memset(&tmap, 0, sizeof(tmap));
+    if constexpr (Shape::TMA) {
+        cudaError_t err = encode_tmap_2d(&tmap, a.logits,
+                                         sizeof(TIn) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                                         (uint64_t)a.M * Shape::TROWS, 128 / sizeof(TIn), 128, 128 / sizeof(TIn),
+                                         R * Shape::TROWS, true);
+        if (err != cudaSuccess) return cuda_fail(err, "cuTensorMapEncodeTiled(logits)");
+    }
+    const int64_t need = (n_oct + kDirectWarps - 1) / kDirectWarps;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const int grid = (int)(need < cap ? need : cap);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3((unsigned)kDirectThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, tmap, a, n_oct);
+    if (err != cudaSuccess) return cuda_fail(err, "direct routing kernel launch");
+    return MOE_OK;
+}
+
+// The direct kernel's shapes: E = 256 or 160, topk <= 8, every group kept or
+// 8 groups.  Returns -1 for other shapes.
+template <typename TIn, int E, int SCORE, bool BIAS>
+int try_direct_e(const RouteArgs& a, cudaStream_t st) {
+    constexpr int GS8 = E / 8;  // experts per group with 8 groups
+    if (a.TG == a.G) {
+        if constexpr (SCORE == kSigmoid && BIAS) return launch_direct<TIn, E, SCORE, BIAS, kKeyApprox, 0>(a, st);
+        else return launch_direct<TIn, E, SCORE, BIAS, kKeyRaw, 0>(a, st);
+    }
+    if (a.G == 8) {
+        constexpr int MODE = SCORE == kSigmoid ? kKeyExact : kKeyRaw;
+        return launch_direct<TIn, E, SCORE, BIAS, MODE, GS8>(a, st);
+    }
+    return -1;
+}
+
+template <typename TIn, int SCORE, bool BIAS>
+int try_direct(const RouteArgs& a, cudaStream_t st) {
+    if (a.K > 8 || !aligned(a.logits, 16)) return -1;
+    // TMA box coordinates are 32-bit: (M * 8) rows of 128 bytes at most
+    if (a.M > (int64_t(1) << 28)) return -1;
+    if (a.E == 256) return try_direct_e<TIn, 256, SCORE, BIAS>(a, st);
+    if (a.E == 160) return try_direct_e<TIn, 160, SCORE, BIAS>(a, st);
+    return -1;
+}
+
 template <typename TIn, int SCORE, bool BIAS>
 int dispatch_typed(const RouteArgs& a, cudaStream_t st) {
     const int E = a.E;
+    {
+        const int rc = try_direct<TIn, SCORE, BIAS>(a, st);
+        if (rc >= 0) return rc;
+    }
     const size_t esz = sizeof(TIn);
     if ((E == 256 || E == 160) && (E == 256 ? 256 / kC256 : 8) % a.G == 0) {
         const int C = (E == 256) ? kC256 : 20;
@@ -307,10 +395,12 @@ int route(const void* logits, int dtype, const float* bias, int64_t M, int E, in
 }  // namespace
 
 int read_routing_watchdog(unsigned int* count) {
-    unsigned int v = 0;
+    unsigned int v = 0, w = 0;
     cudaError_t err = cudaMemcpyFromSymbol(&v, g_watchdog_trips_routing, sizeof(v));
     if (err != cudaSuccess) return cuda_fail(err, "cudaMemcpyFromSymbol(watchdog)");
-    *count = v;
+    err = cudaMemcpyFromSymbol(&w, g_watchdog_trips_direct, sizeof(w));
+    if (err != cudaSuccess) return cuda_fail(err, "cudaMemcpyFromSymbol(direct watchdog)");
+    *count = v + w;
     return MOE_OK;
 }
 

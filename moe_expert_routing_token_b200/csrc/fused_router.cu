@@ -23,6 +23,7 @@
 #include <cstdio>
 #include <mutex>
 #include <type_traits>
+#include <unordered_map>
 
 #include "fused_router.cuh"
 #include "moe_routing.h"
@@ -502,11 +503,12 @@ int launch_fused(const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs
     auto kern = fused_router_kernel<SPLIT, B_MN, BIAS, GRED>;
     {
         static std::mutex mu;
-        static bool done[64] = {};
+        static std::unordered_map<int, bool> done;  // device ordinal -> attributes set
         int dev = 0;
-        cudaGetDevice(&dev);
+        cudaError_t gerr = cudaGetDevice(&dev);
+        if (gerr != cudaSuccess) return set_cuda_error(gerr, "cudaGetDevice");
         std::lock_guard<std::mutex> lk(mu);
-        if (!done[dev & 63]) {
+        if (!done[dev]) {
             cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    (int)fused_smem_bytes());
             if (err != cudaSuccess) return set_cuda_error(err, "cudaFuncSetAttribute(fused router smem)");
@@ -514,7 +516,7 @@ int launch_fused(const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs
                 err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
                 if (err != cudaSuccess) return set_cuda_error(err, "cudaFuncSetAttribute(cluster size)");
             }
-            done[dev & 63] = true;
+            done[dev] = true;
         }
     }
     cudaLaunchConfig_t cfg = {};
@@ -550,9 +552,10 @@ int launch_split(int split, const CUtensorMap& tmA, const CUtensorMap& tmB, cons
 // Largest split whose cluster of one-CTA-per-SM blocks can be scheduled.
 int max_schedulable_split(int dev) {
     static std::mutex mu;
-    static int cached[64] = {};
+    static std::unordered_map<int, int> cached;  // device ordinal -> split
     std::lock_guard<std::mutex> lk(mu);
-    if (cached[dev & 63]) return cached[dev & 63];
+    auto hit = cached.find(dev);
+    if (hit != cached.end()) return hit->second;
     int best = 8;
     auto kern = fused_router_kernel<16, false, true, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem_bytes()) ==
@@ -573,7 +576,7 @@ int max_schedulable_split(int dev) {
         if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) best = 16;
     }
     cudaGetLastError();
-    cached[dev & 63] = best;
+    cached[dev] = best;
     return best;
 }
 
@@ -591,18 +594,19 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 // the first call per device.
 int noalloc_scratch(void** ptr) {
     static std::mutex mu;
-    static void* addr[64] = {};
+    static std::unordered_map<int, void*> addr;  // device ordinal -> address of the array
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return set_cuda_error(err, "cudaGetDevice");
     std::lock_guard<std::mutex> lk(mu);
-    if (addr[dev & 63] == nullptr) {
+    auto hit = addr.find(dev);
+    if (hit == addr.end()) {
         void* p = nullptr;
         err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (err != cudaSuccess) return set_cuda_error(err, "cudaGetSymbolAddress(no-alloc scratch)");
-        addr[dev & 63] = p;
+        hit = addr.emplace(dev, p).first;
     }
-    *ptr = addr[dev & 63];
+    *ptr = hit->second;
     return MOE_OK;
 }
 

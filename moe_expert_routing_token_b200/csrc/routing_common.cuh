@@ -15,6 +15,7 @@ enum Scoring : int { kSoftmax = 0, kSigmoid = 1 };
 enum GroupKind : int { kGroupMax = 0, kGroupTop2Sum = 1 };
 
 constexpr unsigned kFullMask = 0xffffffffu;
+constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s per barrier wait
 
 // Kernel arguments (plain pointers and sizes; identical for every variant).
 struct RouteArgs {
@@ -109,14 +110,45 @@ __device__ __forceinline__ float exp_f32(float x) {
 }
 
 // Logit softcapping of the fused router (routing page §5): c * tanh(x / c),
-// with the accurate tanhf; c = 0 leaves x as it is.  It is strictly
-// increasing, so selection on the raw logits picks the same experts; only the
-// softmax weights and denominators use the capped values.
+// with the accurate tanhf; c = 0 leaves x as it is.  It is monotone, so the
+// experts chosen on the raw logits are also the best by capped value; only
+// the softmax weights and denominators use the capped values.  It is not
+// injective in finite precision: deep in saturation distinct logits cap to
+// one value, and the raw order then picks one member of that tie set.
 __device__ __forceinline__ float softcap_f32(float x, float c) { return c != 0.0f ? c * tanhf(x / c) : x; }
 
 // exp(cap(v) - cap(vmax)), the softmax numerator relative to the row max.
 __device__ __forceinline__ float softmax_num(float v, float vmax, float c) {
     return exp_f32(softcap_f32(v, c) - softcap_f32(vmax, c));
+}
+
+// Bound on |tanh.approx.f32(y) - tanh(y)| used to size the approximate-key
+// band: four times the instruction's documented maximum error of about 2^-11,
+// and checked exhaustively for every bf16 input on the device by the tests.
+constexpr float kTanhApproxErr = 1.0f / 512.0f;
+// Bound on the difference between the paired-reciprocal and the single
+// sigmoid keys (a few fp32 ulp of values below 2).
+constexpr float kPairKeyErr = 1.0f / 1048576.0f;
+
+__device__ __forceinline__ float tanh_approx(float y) {
+    float r;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(y));
+    return r;
+}
+
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// Orderable unsigned key of a score: larger score, larger key.  NaN maps to
+// 1, below every number, and 0 is left for empty slots.
+__device__ __forceinline__ uint32_t order_u32(float v) {
+    uint32_t f = __float_as_uint(v + 0.0f);
+    f = (f & 0x80000000u) ? ~f : (f | 0x80000000u);
+    return (v == v) ? f : 1u;
 }
 
 // Three-input max / min (sm_100).

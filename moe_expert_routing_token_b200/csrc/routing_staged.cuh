@@ -17,7 +17,6 @@
 namespace moe {
 
 constexpr int kStagedWarps = 8;             // consumer warps per block
-constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s per barrier wait
 
 // Incremented when a barrier wait times out (a kernel then stops early and
 // leaves its outputs unspecified); read back by moe_watchdog_trips().

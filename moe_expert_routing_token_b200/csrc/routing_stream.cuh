@@ -47,35 +47,6 @@ constexpr int kStreamP2Warps = 8;    // phase-2 warps (block it goes to warp it 
 constexpr int kStreamRows = 32;      // rows per stage (= lanes of a phase-2 warp)
 constexpr int kStreamThreads = (1 + kStreamTeams * kStreamTeamWarps + kStreamP2Warps) * 32;
 constexpr int kTabStride = 12;     // u32 words per row of the candidate table (48 B)
-// Bound on |tanh.approx.f32(y) - tanh(y)| used to size the approximate-key
-// band: four times the instruction's documented maximum error of about 2^-11,
-// and checked exhaustively for every bf16 input on the device by the tests.
-constexpr float kTanhApproxErr = 1.0f / 512.0f;
-// Bound on the difference between the paired-reciprocal and the single
-// sigmoid keys (a few fp32 ulp of values below 2).
-constexpr float kPairKeyErr = 1.0f / 1048576.0f;
-
-__device__ __forceinline__ float tanh_approx(float y) {
-    float r;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(y));
-    return r;
-}
-
-__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
-                                                   unsigned long long c) {
-    unsigned long long r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
-// Orderable unsigned key of a score: larger score, larger key.  NaN maps to
-// 1, below every number, and 0 is left for empty slots.
-__device__ __forceinline__ uint32_t order_u32(float v) {
-    uint32_t f = __float_as_uint(v + 0.0f);
-    f = (f & 0x80000000u) ? ~f : (f | 0x80000000u);
-    return (v == v) ? f : 1u;
-}
-
 // Insert (v, e) into the descending list kk/ii.  Candidates arrive in
 // ascending index order, so the strict comparison keeps equal keys in index
 // order.

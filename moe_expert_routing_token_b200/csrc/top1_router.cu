@@ -7,9 +7,13 @@
 //   id   = arg-max_e l_e               lowest index among equal logits
 //   w    = 1 / sum_e exp(cap_e - cap_id)   the page's invsumexp
 //
-// The arg-max is taken on the raw logits: c * tanh(x / c) is strictly
-// increasing, so the expert is the same, and the fp32 tanh cannot merge two
-// distinct logits into one capped value.
+// The arg-max is taken on the raw logits.  c * tanh(x / c) is monotone, so
+// the raw maximum is also a maximum of the capped values, but it is not
+// injective in finite precision: far in the saturated range (|x / c| above
+// about 9 in fp32, 19 in double) distinct logits cap to the same value.  Such
+// a row has several equal largest capped values; the raw arg-max is one of
+// them, and the weight, which depends only on the capped values, is the same
+// whichever of them is chosen.
 //
 // With E <= 8 experts the work is 2 * E flops per 2-byte hidden value, below
 // the B200's fp32 CUDA-core ridge (about 11 flops per byte), so one kernel

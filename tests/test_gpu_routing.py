@@ -13,7 +13,7 @@ import torch
 import moe_expert_routing_token_b200 as moe
 import oracle
 from moe_expert_routing_token_b200 import inputs
-from tests import parity
+from oracle import parity
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -269,6 +269,28 @@ def test_softcapped_softmax(M, E, G, TG, k, renorm, dtype):
                          fp32_logits=(dtype == torch.float32),
                          w_rtol=2e-5 if dtype == torch.float32 else None)
     assert rep.ok(), rep.summary()
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (256, 8)])
+def test_softcap_saturated_ties(E, k):
+    """c = 1 and logits far into tanh's saturation: 20, 25 and 30 (and, at
+    E = 256, a block of 24 logits in [20, 40]) all cap to exactly 1.  The kernels select
+    on the raw logits, the oracle on the capped values with ties to the lower
+    index; the rows must count as near ties and pass."""
+    M = 64
+    x = inputs.random_logits(M, E, 1.0, torch.float32, seed=E)
+    x[:, 1] = 20.0
+    x[:, 3] = 25.0
+    x[:, 5] = 30.0  # k + 1 saturated values at E = 8: the k-th pick is tied
+    if E == 256:
+        x[:, 100:124] = torch.linspace(20.0, 40.0, 24)
+    w, ids = moe.grouped_topk(x.to(DEV), k, True, 1, 1, 1.0, softcap=1.0)
+    torch.cuda.synchronize()
+    orc = oracle.grouped_topk(oracle.softcap_logits(x, 1.0), k, True, 1, 1, 1.0)
+    rep = parity.compare(w.cpu().numpy(), ids.cpu().numpy(), orc, E=E, G=1, TG=1, k=k, renorm=True, rsf=1.0,
+                         fp32_logits=True, w_rtol=2e-5)
+    assert rep.ok(), rep.summary()
+    assert rep.near_tie == M, rep.summary()
 
 
 def test_softcap_zero_is_the_plain_call():

@@ -29,7 +29,7 @@ from tests.test_gpu_routing import check
 
 pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
-HEADER = os.path.join(HERE, "..", "moe_expert_routing_token_b200", "csrc", "routing_stream.cuh")
+HEADER = os.path.join(HERE, "..", "moe_expert_routing_token_b200", "csrc", "routing_common.cuh")
 
 
 def _header_constant(name):
