@@ -16,9 +16,15 @@ Timing: inputs are resident in HBM before the timed region; every step reads a
 different buffer of a rotating pool larger than L2, so reads come from DRAM.
 The K steps are replayed from CUDA graphs (exactly K launches of the routing
 kernel) and timed with CUDA events on the launching stream, bracketed by a
-barrier and a device synchronise; the job time is the max over ranks.  Under
-torchrun each rank routes its own batches (no data-path collective: rows are
-independent), so scaling is weak.
+barrier and a device synchronise; the job time is the max over ranks.  A
+short GPU sleep is queued before the start event so that the host's graph
+launch is not inside the timed region.  Under torchrun each rank routes its
+own batches (no data-path collective: rows are independent), so scaling is
+weak.
+
+On one GPU the line also carries ``per_config``: every workload size the
+routing spec names, timed cold (rotating pool) and hot (one buffer), with a
+parity sample against the oracle taken in the CPU-baseline leg.
 """
 from __future__ import annotations
 
@@ -48,10 +54,20 @@ WORKLOAD_METRICS = {
 
 def metric_for(name: str) -> str:
     return WORKLOAD_METRICS.get(name, METRIC)
+
+
 L2_BYTES = 126 * 1024 * 1024
+ROUTING = ("sigmoid", "biased", "grouped", "softmax")
+# Every size the routing spec quotes (the workload, M): the per-config table.
+PER_CONFIG = [("softmax", 64), ("sigmoid", 1), ("sigmoid", 16), ("sigmoid", 64), ("sigmoid", 256),
+              ("sigmoid", 4096), ("sigmoid", 16384), ("biased", 4096), ("biased", 32), ("grouped", 16384),
+              ("fused", 8192), ("fused", 64), ("top1", 8192)]
+# GPU sleep queued before the start event: about 100 us at the B200's clocks,
+# longer than the host needs to submit the first graph of the timed region.
+SLEEP_CYCLES = 200_000
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=48000)
@@ -62,9 +78,11 @@ def parse_args():
     ap.add_argument("--M", type=int, default=None, help="tokens per step (default: workload's)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--per-config-steps", type=int, default=1000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-soak", action="store_true", help="skip the 1 s clock-sampling soak")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 DEFAULT_M = {"sigmoid": 16384, "biased": 4096, "grouped": 16384, "softmax": 64, "fused": 8192, "top1": 8192,
@@ -152,6 +170,19 @@ def profiled_traffic(name: str, M: int):
     return float(val.group(1))
 
 
+def host_cpu() -> dict:
+    """The host the CPU baseline runs on: core count and model name."""
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
 # ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
@@ -203,7 +234,9 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle timing (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
-def oracle_call(name: str, d: dict, rows: slice):
+def oracle_call(name: str, d: dict, rows):
+    """The oracle on the rows ``rows`` (a slice or an index array) of workload
+    input ``d``."""
     import oracle
     sp = d["spec"]
     if name == "top1":
@@ -235,9 +268,9 @@ def time_oracle(name: str, M: int, seconds: float) -> dict:
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return {"value": n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens ({n // rows} x {rows}-token batches of the {name} workload, "
-                      f"M={M} draw), single-threaded C oracle in double, {el:.1f} s"}
+    return dict({"value": n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                 "sample": f"{n} tokens ({n // rows} x {rows}-token batches of the {name} workload, "
+                           f"M={M} draw), single-threaded C oracle in double, {el:.1f} s"}, **host_cpu())
 
 
 # ---------------------------------------------------------------------------
@@ -289,8 +322,8 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{rows} of {M} tokens per step"},
+            "cpu_baseline": dict({"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                  "sample": f"{rows} of {M} tokens per step"}, **host_cpu()),
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -308,11 +341,242 @@ def _oracle_row_time(name, d):
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
+class Workload:
+    """Device buffers and the C-ABI call of one workload at one size: a pool
+    of input/output sets whose total exceeds 4x L2 (``rotate``), or one set."""
+
+    def __init__(self, name: str, M: int, dev, seed: int, rotate: bool = True, d=None):
+        import torch
+
+        from moe_expert_routing_token_b200 import inputs, routing
+        self.name, self.M, self.dev = name, M, dev
+        self.lib = routing.lib()
+        self.sp = sp = inputs.SPECS[name]
+        self.d = d = inputs.make(name, M, seed=seed) if d is None else d
+        self.per_set = algorithmic_bytes(name, M)
+        self.pool = max(2, min(256, -(-4 * L2_BYTES // self.per_set))) if rotate else 1
+        if name in ("fused", "top1"):
+            src = d["hidden"].to(dev)
+            self.wgt = d["weight"].to(dev)
+        else:
+            src = d["logits"].to(dev)
+        self.xs = [src] + [src.clone() for _ in range(self.pool - 1)]
+        self.bias = d["bias"].to(dev) if d["bias"] is not None else None
+        self.ws = [torch.empty(M, sp.topk, dtype=torch.float32, device=dev) for _ in range(self.pool)]
+        self.ids = [torch.empty(M, sp.topk, dtype=torch.int32, device=dev) for _ in range(self.pool)]
+        self.wsp_bytes = routing.fused_router_workspace_size(M, sp.K, sp.E) if name == "fused" else 0
+        self.wsp = [torch.zeros(max(1, self.wsp_bytes), dtype=torch.uint8, device=dev) for _ in range(self.pool)]
+        self.dcode = routing.MOE_DTYPE_BF16 if sp.dtype == torch.bfloat16 else routing.MOE_DTYPE_F32
+        self.launches_per_call = 1
+
+    def call(self, i: int, stream_ptr: int, logits_out=None):
+        from moe_expert_routing_token_b200 import routing
+        lib, sp, M, name = self.lib, self.sp, self.M, self.name
+        j = i % self.pool
+        bptr = self.bias.data_ptr() if self.bias is not None else None
+        lptr = logits_out.data_ptr() if logits_out is not None else None
+        if name == "fused":
+            st = lib.moe_fused_router_topk(self.xs[j].data_ptr(), self.wgt.data_ptr(), routing.MOE_WEIGHT_K_BY_E,
+                                           bptr, M, sp.K, sp.E, sp.topk, int(sp.renormalize),
+                                           sp.num_expert_group, sp.topk_group, sp.routed_scaling_factor,
+                                           self.ws[j].data_ptr(), self.ids[j].data_ptr(), lptr,
+                                           self.wsp[j].data_ptr() if self.wsp_bytes else None, self.wsp_bytes,
+                                           stream_ptr)
+        elif name == "top1":
+            st = lib.moe_fused_router_top1(self.xs[j].data_ptr(), self.wgt.data_ptr(), routing.MOE_WEIGHT_E_BY_K,
+                                           M, sp.K, sp.E, sp.softcap, self.ws[j].data_ptr(), self.ids[j].data_ptr(),
+                                           lptr, stream_ptr)
+        elif name in ("softmax", "grouped"):
+            st = lib.moe_grouped_topk(self.xs[j].data_ptr(), self.dcode, M, sp.E, sp.topk, int(sp.renormalize),
+                                      sp.num_expert_group, sp.topk_group, sp.routed_scaling_factor,
+                                      self.ws[j].data_ptr(), self.ids[j].data_ptr(), stream_ptr)
+        else:
+            st = lib.moe_biased_grouped_topk(self.xs[j].data_ptr(), self.dcode, bptr, M, sp.E, sp.topk,
+                                             int(sp.renormalize), sp.num_expert_group, sp.topk_group,
+                                             sp.routed_scaling_factor, self.ws[j].data_ptr(),
+                                             self.ids[j].data_ptr(), stream_ptr)
+        if st != 0:
+            raise RuntimeError(lib.moe_last_error().decode())
+
+
+class GraphTimer:
+    """CUDA graphs of consecutive calls of one workload - a whole number of
+    passes over its buffer pool, at least 64 calls - and of the remainders,
+    replayed for exactly n steps and timed with CUDA events on the launching
+    stream."""
+
+    def __init__(self, call, pool: int, steps: int, warmup: int, stream):
+        import torch
+        self.stream = stream
+        self.pool = pool = pool * max(1, -(-64 // pool))  # calls per graph
+        sptr = stream.cuda_stream
+
+        def capture(nsteps: int):
+            if nsteps == 0:
+                return None
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(nsteps):
+                    call(i, sptr)
+            return g
+
+        for i in range(3):  # eager warm-up of the C ABI (first-call set-up happens here)
+            call(i, sptr)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            self.g_pool = capture(pool)
+            self.g_rem = {steps % pool: capture(steps % pool), warmup % pool: capture(warmup % pool)}
+
+    def run(self, n: int):
+        for _ in range(n // self.pool):
+            self.g_pool.replay()
+        g = self.g_rem.get(n % self.pool)
+        if g is not None:
+            g.replay()
+
+    def time_ms(self, n: int, barrier=None) -> float:
+        """Device time of exactly n steps: synchronise (and barrier), queue a
+        GPU sleep that covers the host's graph submission, then events around
+        the n steps."""
+        import torch
+        if barrier is not None:
+            barrier()
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            torch.cuda._sleep(SLEEP_CYCLES)
+            start.record(self.stream)
+            self.run(n)
+            stop.record(self.stream)
+        torch.cuda.synchronize()
+        if barrier is not None:
+            barrier()
+        return start.elapsed_time(stop)
+
+    def release(self):
+        self.g_pool = None
+        self.g_rem = {}
+
+
+def roofline(name: str, M: int, us_per_call: float, clocks, peaks) -> dict:
+    from moe_expert_routing_token_b200 import inputs
+    sp = inputs.SPECS[name]
+    if name == "fused":
+        flops = 2.0 * M * sp.K * sp.E
+        achieved = flops / (us_per_call * 1e-6) / 1e12
+        # A long loop of GEMMs runs under the power cap: then the sustained
+        # cuBLAS figure is the comparable peak, else the burst one.
+        capped = bool(clocks) and ("sw_power_cap" in clocks.get("reasons", []) or
+                                   clocks.get("sm_mhz", 0) < 0.9 * clocks.get("sm_max_mhz", 1))
+        if capped and peaks.get("bf16_tflops_sustained"):
+            peak, kind = peaks["bf16_tflops_sustained"], "bf16 sustained (run under the power cap)"
+        else:
+            peak, kind = peaks["bf16_tflops"], "bf16 burst"
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(name, M),
+                "algorithmic_flops_per_launch": flops, "peak_source": f"{peaks['source']} {kind}"}
+    per_set = algorithmic_bytes(name, M)
+    achieved = per_set / (us_per_call * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(name, M),
+            "algorithmic_bytes_per_launch": per_set, "peak_source": f"{peaks['source']} HBM copy"}
+
+
+def sample_rows(M: int, n: int):
+    """Rows for a parity sample: all rows when M <= n, else the first and the
+    last n / 2 rows (the last covers the ragged tail of the grid)."""
+    import numpy as np
+    if M <= n:
+        return np.arange(M)
+    h = n // 2
+    return np.concatenate([np.arange(h), np.arange(M - (n - h), M)])
+
+
+def parity_sample(wl: Workload, stream) -> dict:
+    """CPU-baseline leg: the oracle on a sample of the workload's rows against
+    the GPU's outputs for them (the inputs of every pool slot are the same
+    draw).  Fused and top-1 routers: one extra untimed call returns the fp32
+    logits, the oracle routes those (the routing step, bit-exact rules) and the
+    logits are checked against the oracle's double-precision projection."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from oracle import parity
+    name, M, sp, d = wl.name, wl.M, wl.sp, wl.d
+    n = {"fused": 64, "top1": 512}.get(name, 2048)
+    rows = sample_rows(M, n)
+    out = {"rows": int(len(rows))}
+    logits = None
+    if name in ("fused", "top1"):
+        logits = torch.empty(M, sp.E, dtype=torch.float32, device=wl.dev)
+        wl.call(0, stream.cuda_stream, logits_out=logits)
+    torch.cuda.synchronize()
+    w = wl.ws[0].cpu().numpy()[rows]
+    ids = wl.ids[0].cpu().numpy()[rows]
+    if name in ROUTING:
+        orc = oracle_call(name, d, rows)
+        rep = parity.compare(w, ids, orc, E=sp.E, G=sp.num_expert_group, TG=sp.topk_group, k=sp.topk,
+                             renorm=sp.renormalize, rsf=sp.routed_scaling_factor,
+                             fp32_logits=(sp.dtype == torch.float32))
+    elif name == "fused":
+        lg = logits.cpu().double().numpy()[rows]
+        ref = oracle.router_logits(d["hidden"][rows], d["weight"], weight_layout=0)
+        out["max_logit_err"] = float(np.abs(lg - ref).max())
+        orc = oracle.biased_grouped_topk(lg, d["bias"], sp.topk, sp.renormalize, sp.num_expert_group,
+                                         sp.topk_group, sp.routed_scaling_factor)
+        rep = parity.compare(w, ids, orc, E=sp.E, G=sp.num_expert_group, TG=sp.topk_group, k=sp.topk,
+                             renorm=sp.renormalize, rsf=sp.routed_scaling_factor, fp32_logits=False)
+    else:
+        lg = logits.cpu().double().numpy()[rows]
+        ref = oracle.router_logits(d["hidden"][rows], d["weight"], weight_layout=1)
+        out["max_logit_err"] = float(np.abs(lg - ref).max())
+        orc = oracle.topk_softmax(oracle.softcap_logits(lg, sp.softcap), 1, False)
+        rep = parity.compare(w, ids, orc, E=sp.E, G=1, TG=1, k=1, renorm=False, rsf=1.0, fp32_logits=True,
+                             w_rtol=2e-5)
+    out.update({"near_tie": rep.near_tie, "max_weight_err": rep.max_weight_err, "ok": rep.ok(),
+                "checked_by": "oracle on the sampled rows (CPU-baseline leg)"})
+    if not rep.ok():
+        out["failures"] = rep.failures[:4]
+    return out
+
+
+def run_per_config(dev, stream, steps: int, peaks, with_parity: bool) -> list:
+    """Every size the routing spec names: cold (rotating pool > 4x L2) and hot
+    (one buffer) device time per call, roofline fraction, parity sample."""
+    import torch
+    rows = []
+    for name, M in PER_CONFIG:
+        from moe_expert_routing_token_b200 import inputs
+        seed = inputs.default_seed(name, M)
+        entry = {"workload": name, "M": M}
+        d = inputs.make(name, M, seed=seed)
+        for kind, rotate in (("cold", True), ("hot", False)):
+            wl = Workload(name, M, dev, seed, rotate=rotate, d=d)
+            gt = GraphTimer(wl.call, wl.pool, steps, 3, stream)
+            gt.run(3)
+            ms = gt.time_ms(steps)
+            entry[f"us_per_call_{kind}"] = ms * 1e3 / steps
+            if kind == "cold":
+                entry["pool_sets"] = wl.pool
+                entry["tokens_per_s"] = M * steps / (ms / 1e3)
+                rf = roofline(name, M, entry["us_per_call_cold"], None, peaks)
+                entry["roofline"] = {k: rf[k] for k in ("bound", "achieved", "peak", "unit", "frac")}
+                if with_parity:
+                    entry["parity"] = parity_sample(wl, stream)
+            gt.release()
+            del wl
+            torch.cuda.synchronize()
+        rows.append(entry)
+    return rows
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from moe_expert_routing_token_b200 import build, inputs, routing
+    from moe_expert_routing_token_b200 import build, routing
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -330,104 +594,24 @@ def run_ours(args):
         build.build()
     if world > 1:
         dist.barrier()
-    lib = routing.lib()
+    routing.lib()
 
     name = args.workload
     M = args.M or DEFAULT_M[name]
-    sp = inputs.SPECS[name]
-    d = inputs.make(name, M, seed=rank_seed(name, M, rank))
     # a dedicated stream: graphs cannot be captured on the legacy default stream
     stream = torch.cuda.Stream(dev)
     torch.cuda.set_stream(stream)
-    sptr = stream.cuda_stream
 
-    # ---- rotating device pool larger than L2 --------------------------------
-    per_set = algorithmic_bytes(name, M)
-    pool = max(2, min(256, -(-4 * L2_BYTES // per_set)))
-    if name in ("fused", "top1"):
-        src_x = d["hidden"].to(dev)
-        wgt = d["weight"].to(dev)
-    else:
-        src_x = d["logits"].to(dev)
-    xs = [src_x.clone() for _ in range(pool)]
-    bias = d["bias"].to(dev) if d["bias"] is not None else None
-    bptr = bias.data_ptr() if bias is not None else None
-    ws = [torch.empty(M, sp.topk, dtype=torch.float32, device=dev) for _ in range(pool)]
-    ids = [torch.empty(M, sp.topk, dtype=torch.int32, device=dev) for _ in range(pool)]
-    wsp_bytes = routing.fused_router_workspace_size(M, sp.K, sp.E) if name == "fused" else 0
-    wsp = [torch.zeros(max(1, wsp_bytes), dtype=torch.uint8, device=dev) for _ in range(pool)]
-
-    dcode = routing.MOE_DTYPE_BF16 if sp.dtype == torch.bfloat16 else routing.MOE_DTYPE_F32
-
-    def call(i: int):
-        j = i % pool
-        if name == "fused":
-            st = lib.moe_fused_router_topk(xs[j].data_ptr(), wgt.data_ptr(), routing.MOE_WEIGHT_K_BY_E,
-                                           bptr, M, sp.K, sp.E, sp.topk, int(sp.renormalize),
-                                           sp.num_expert_group, sp.topk_group,
-                                           sp.routed_scaling_factor, ws[j].data_ptr(),
-                                           ids[j].data_ptr(), None,
-                                           wsp[j].data_ptr() if wsp_bytes else None, wsp_bytes, sptr)
-        elif name == "top1":
-            st = lib.moe_fused_router_top1(xs[j].data_ptr(), wgt.data_ptr(), routing.MOE_WEIGHT_E_BY_K, M, sp.K,
-                                           sp.E, sp.softcap, ws[j].data_ptr(), ids[j].data_ptr(), None, sptr)
-        elif name in ("softmax", "grouped"):
-            st = lib.moe_grouped_topk(xs[j].data_ptr(), dcode, M, sp.E, sp.topk, int(sp.renormalize),
-                                      sp.num_expert_group, sp.topk_group, sp.routed_scaling_factor,
-                                      ws[j].data_ptr(), ids[j].data_ptr(), sptr)
-        else:
-            st = lib.moe_biased_grouped_topk(xs[j].data_ptr(), dcode, bptr, M, sp.E, sp.topk,
-                                             int(sp.renormalize), sp.num_expert_group,
-                                             sp.topk_group, sp.routed_scaling_factor,
-                                             ws[j].data_ptr(), ids[j].data_ptr(), sptr)
-        if st != 0:
-            raise RuntimeError(lib.moe_last_error().decode())
-
-    # ---- graphs: one of `pool` steps and one of the remainder -----------------
-    for i in range(3):  # eager warm-up of the C ABI (first-call set-up happens here)
-        call(i)
-    torch.cuda.synchronize()
-
-    def capture(nsteps: int):
-        if nsteps == 0:
-            return None
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(nsteps):
-                call(i)
-        return g
-
-    with torch.cuda.stream(stream):
-        g_pool = capture(pool)
-        g_rem = capture(args.steps % pool)
-        g_warm_rem = capture(args.warmup % pool)
-
-    def run_steps(n: int, rem_graph):
-        for _ in range(n // pool):
-            g_pool.replay()
-        if rem_graph is not None:
-            rem_graph.replay()
-
+    wl = Workload(name, M, dev, rank_seed(name, M, rank))
+    gt = GraphTimer(wl.call, wl.pool, args.steps, args.warmup, stream)
     sampler = ClockSampler(local_rank) if rank == 0 else None
-    run_steps(args.warmup, g_warm_rem)
+    gt.run(args.warmup)
     # untimed soak so that the clock sampler sees the GPU under this load
     t_soak = time.time()
     while not args.no_soak and time.time() - t_soak < 1.0:
-        g_pool.replay()
+        gt.g_pool.replay()
         torch.cuda.synchronize()
-
-    start = torch.cuda.Event(enable_timing=True)
-    stop = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    run_steps(args.steps, g_rem)
-    stop.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms = start.elapsed_time(stop)
+    ms = gt.time_ms(args.steps, barrier=dist.barrier if world > 1 else None)
     clocks = sampler.stop() if sampler else None
     ms = job_elapsed_ms(ms, world, dev)
     value = job_tokens_per_s(M, args.steps, world, ms)
@@ -436,7 +620,7 @@ def run_ours(args):
     # ---- end to end through the public API with host buffers ----------------
     e2e = None
     if not args.no_e2e:
-        e2e = e2e_measure(name, M, sp, d, dev, stream, world, args)
+        e2e = e2e_measure(name, M, wl.sp, wl.d, dev, stream, world, args)
 
     peaks = measured_peaks()
     line = {"metric": metric_for(name), "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -444,37 +628,26 @@ def run_ours(args):
             "us_per_call": us_per_call, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": dict(workload_desc(name, M), parallelism=f"dp{world} (rows sharded, no collective)",
-                           l2=(f"rotating pool of {pool} input/output sets, "
-                               f"{pool * per_set / 2**20:.0f} MiB > 126 MiB L2"),
-                           timing="CUDA graphs of the C-ABI calls, CUDA events on the launch stream"),
-            "gpu_launches": args.steps,
-            "clocks": clocks}
-    if name == "fused":
-        flops = 2.0 * M * sp.K * sp.E
-        achieved = flops / (us_per_call * 1e-6) / 1e12
-        # A long loop of GEMMs runs under the power cap: then the sustained
-        # cuBLAS figure is the comparable peak, else the burst one.
-        capped = bool(clocks) and ("sw_power_cap" in clocks.get("reasons", []) or
-                                   clocks.get("sm_mhz", 0) < 0.9 * clocks.get("sm_max_mhz", 1))
-        if capped and peaks.get("bf16_tflops_sustained"):
-            peak, kind = peaks["bf16_tflops_sustained"], "bf16 sustained (run under the power cap)"
-        else:
-            peak, kind = peaks["bf16_tflops"], "bf16 burst"
-        line["roofline"] = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                            "frac": achieved / peak, "traffic": profiled_traffic(name, M),
-                            "peak_source": f"{peaks['source']} {kind}"}
-    else:
-        achieved = per_set / (us_per_call * 1e-6) / 1e9
-        peak = peaks["hbm_gbs"]
-        line["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                            "frac": achieved / peak, "traffic": profiled_traffic(name, M),
-                            "algorithmic_bytes_per_launch": per_set,
-                            "peak_source": f"{peaks['source']} HBM copy"}
+                           l2=(f"rotating pool of {wl.pool} input/output sets, "
+                               f"{wl.pool * wl.per_set / 2**20:.0f} MiB > 126 MiB L2"),
+                           timing=("CUDA graphs of the C-ABI calls, CUDA events on the launch stream; "
+                                   "a GPU sleep before the start event covers the host's graph launch")),
+            "gpu_launches": args.steps * wl.launches_per_call,
+            "clocks": clocks,
+            "roofline": roofline(name, M, us_per_call, clocks, peaks)}
     line["e2e"] = e2e
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if with_cpu:
         line["cpu_baseline"] = time_oracle(name, M, args.cpu_seconds)
+        p = parity_sample(wl, stream)
+        line["near_tie"] = p["near_tie"]
+        line["max_weight_err"] = p["max_weight_err"]
+        line["parity_sample"] = p
+    gt.release()
+    del wl
+    if world == 1 and not args.no_per_config:
+        line["per_config"] = run_per_config(dev, stream, args.per_config_steps, peaks, with_cpu)
     if world > 1:
-        del g_pool, g_rem, g_warm_rem
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -488,7 +661,6 @@ def e2e_measure(name, M, sp, d, dev, stream, world, args):
     import torch.distributed as dist
 
     from moe_expert_routing_token_b200 import routing
-    lib = routing.lib()
     steps = max(1, min(args.steps, 200))
     src = (d["hidden"] if name in ("fused", "top1") else d["logits"]).pin_memory()
     x = torch.empty_like(src, device=dev)
@@ -569,15 +741,51 @@ def time_perm_oracle(M: int, seconds: float) -> dict:
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return {"value": n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens ({n // M} x {M}-token batches), single-threaded C oracle, {el:.1f} s"}
+    return dict({"value": n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                 "sample": f"{n} tokens ({n // M} x {M}-token batches), single-threaded C oracle, {el:.1f} s"},
+                **host_cpu())
+
+
+class PermWorkload:
+    """Device buffers and the C-ABI call of the expert permutation."""
+
+    def __init__(self, M: int, dev, seed: int):
+        import torch
+
+        from moe_expert_routing_token_b200 import inputs, routing
+        self.M, self.n = M, M * PERM_K
+        self.lib = routing.lib()
+        self.ids_h, self.w_h = inputs.routed_ids(M, PERM_K, PERM_E, seed=seed)
+        self.per_set = perm_bytes(M)
+        self.pool = max(2, min(256, -(-4 * L2_BYTES // self.per_set)))
+        self.ids = [self.ids_h.to(dev) for _ in range(self.pool)]
+        self.wts = [self.w_h.to(dev) for _ in range(self.pool)]
+        n = self.n
+        self.outs = [[torch.empty(PERM_E, dtype=torch.int32, device=dev),
+                      torch.empty(PERM_E + 1, dtype=torch.int32, device=dev),
+                      torch.empty(n, dtype=torch.int32, device=dev), torch.empty(n, dtype=torch.int32, device=dev),
+                      torch.empty(n, dtype=torch.float32, device=dev)] for _ in range(self.pool)]
+        self.wsb = routing.expert_permutation_workspace_size(M, PERM_K, PERM_E)
+        self.wsp = [torch.empty(max(1, self.wsb), dtype=torch.uint8, device=dev) for _ in range(self.pool)]
+
+    def call(self, i: int, stream_ptr: int, src_ids=None, src_w=None, out=None, ws=None):
+        j = i % self.pool
+        o = out if out is not None else self.outs[j]
+        st = self.lib.moe_expert_permutation((src_ids if src_ids is not None else self.ids[j]).data_ptr(),
+                                             (src_w if src_w is not None else self.wts[j]).data_ptr(), self.M,
+                                             PERM_K, PERM_E, o[0].data_ptr(), o[1].data_ptr(), o[2].data_ptr(),
+                                             o[3].data_ptr(), o[4].data_ptr(),
+                                             (ws if ws is not None else self.wsp[j]).data_ptr(), self.wsb,
+                                             stream_ptr)
+        if st != 0:
+            raise RuntimeError(self.lib.moe_last_error().decode())
 
 
 def run_permute(args):
     import torch
     import torch.distributed as dist
 
-    from moe_expert_routing_token_b200 import build, inputs, routing
+    from moe_expert_routing_token_b200 import build, routing
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -607,75 +815,19 @@ def run_permute(args):
         build.build()
     if world > 1:
         dist.barrier()
-    lib = routing.lib()
+    routing.lib()
     M = args.M or DEFAULT_M["permute"]
-    n = M * PERM_K
-    ids_h, w_h = inputs.routed_ids(M, PERM_K, PERM_E, seed=rank_seed("sigmoid", M, rank))
     stream = torch.cuda.Stream(dev)
     torch.cuda.set_stream(stream)
-    sptr = stream.cuda_stream
-    per_set = perm_bytes(M)
-    pool = max(2, min(256, -(-4 * L2_BYTES // per_set)))
-    ids = [ids_h.to(dev) for _ in range(pool)]
-    wts = [w_h.to(dev) for _ in range(pool)]
-    outs = [[torch.empty(PERM_E, dtype=torch.int32, device=dev), torch.empty(PERM_E + 1, dtype=torch.int32, device=dev),
-             torch.empty(n, dtype=torch.int32, device=dev), torch.empty(n, dtype=torch.int32, device=dev),
-             torch.empty(n, dtype=torch.float32, device=dev)] for _ in range(pool)]
-    wsb = routing.expert_permutation_workspace_size(M, PERM_K, PERM_E)
-    wsp = [torch.empty(max(1, wsb), dtype=torch.uint8, device=dev) for _ in range(pool)]
-
-    def call(i: int, src_ids=None, src_w=None, out=None, ws=None):
-        j = i % pool
-        o = out if out is not None else outs[j]
-        st = lib.moe_expert_permutation((src_ids if src_ids is not None else ids[j]).data_ptr(),
-                                        (src_w if src_w is not None else wts[j]).data_ptr(), M, PERM_K, PERM_E,
-                                        o[0].data_ptr(), o[1].data_ptr(), o[2].data_ptr(), o[3].data_ptr(),
-                                        o[4].data_ptr(), (ws if ws is not None else wsp[j]).data_ptr(), wsb, sptr)
-        if st != 0:
-            raise RuntimeError(lib.moe_last_error().decode())
-
-    for i in range(3):
-        call(i)
-    torch.cuda.synchronize()
-
-    def capture(nsteps: int):
-        if nsteps == 0:
-            return None
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(nsteps):
-                call(i)
-        return g
-
-    with torch.cuda.stream(stream):
-        g_pool = capture(pool)
-        g_rem = capture(args.steps % pool)
-        g_warm_rem = capture(args.warmup % pool)
-
-    def run_steps(nst: int, rem_graph):
-        for _ in range(nst // pool):
-            g_pool.replay()
-        if rem_graph is not None:
-            rem_graph.replay()
-
+    pw = PermWorkload(M, dev, rank_seed("sigmoid", M, rank))
+    gt = GraphTimer(pw.call, pw.pool, args.steps, args.warmup, stream)
     sampler = ClockSampler(local_rank) if rank == 0 else None
-    run_steps(args.warmup, g_warm_rem)
+    gt.run(args.warmup)
     t_soak = time.time()
     while not args.no_soak and time.time() - t_soak < 1.0:
-        g_pool.replay()
+        gt.g_pool.replay()
         torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    stop = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    run_steps(args.steps, g_rem)
-    stop.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms = job_elapsed_ms(start.elapsed_time(stop), world, dev)
+    ms = job_elapsed_ms(gt.time_ms(args.steps, barrier=dist.barrier if world > 1 else None), world, dev)
     clocks = sampler.stop() if sampler else None
     value = job_tokens_per_s(M, args.steps, world, ms)
     us_per_call = ms * 1e3 / args.steps
@@ -683,17 +835,17 @@ def run_permute(args):
     e2e = None
     if not args.no_e2e:
         # host buffers in, permutation out, every step
-        h_ids = ids_h.pin_memory()
-        h_w = w_h.pin_memory()
-        h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs[0]]
-        d_ids, d_w = ids[0], wts[0]
+        h_ids = pw.ids_h.pin_memory()
+        h_w = pw.w_h.pin_memory()
+        h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in pw.outs[0]]
+        d_ids, d_w = pw.ids[0], pw.wts[0]
         steps = 200
 
         def step():
             d_ids.copy_(h_ids, non_blocking=True)
             d_w.copy_(h_w, non_blocking=True)
-            call(0, d_ids, d_w, outs[0], wsp[0])
-            for h, d in zip(h_out, outs[0]):
+            pw.call(0, stream.cuda_stream, d_ids, d_w, pw.outs[0], pw.wsp[0])
+            for h, d in zip(h_out, pw.outs[0]):
                 h.copy_(d, non_blocking=True)
 
         with torch.cuda.stream(stream):
@@ -711,28 +863,29 @@ def run_permute(args):
             torch.cuda.synchronize()
         ems = job_elapsed_ms(a.elapsed_time(b), world, dev)
         e2e = {"value": job_tokens_per_s(M, steps, world, ems), "unit": "tokens/s",
-               "h2d_bytes_per_step": n * 8, "d2h_bytes_per_step": sum(t.numel() * 4 for t in h_out),
+               "h2d_bytes_per_step": pw.n * 8, "d2h_bytes_per_step": sum(t.numel() * 4 for t in h_out),
                "steps": steps}
 
     peaks = measured_peaks()
-    achieved = per_set / (us_per_call * 1e-6) / 1e9
+    achieved = pw.per_set / (us_per_call * 1e-6) / 1e9
     line = {"metric": PERM_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
             "us_per_call": us_per_call, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int32", "data": "synthetic",
             "config": dict(perm_desc(M), parallelism=f"dp{world} (rows sharded, no collective)",
-                           l2=f"rotating pool of {pool} sets, {pool * per_set / 2**20:.0f} MiB > 126 MiB L2",
-                           timing="CUDA graphs of the C-ABI calls, CUDA events on the launch stream"),
+                           l2=f"rotating pool of {pw.pool} sets, {pw.pool * pw.per_set / 2**20:.0f} MiB > 126 MiB L2",
+                           timing=("CUDA graphs of the C-ABI calls, CUDA events on the launch stream; "
+                                   "a GPU sleep before the start event covers the host's graph launch")),
             "gpu_launches": 3 * args.steps, "clocks": clocks,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                         "algorithmic_bytes_per_launch": per_set,
+                         "algorithmic_bytes_per_launch": pw.per_set,
                          "peak_source": f"{peaks['source']} HBM copy"},
             "e2e": e2e}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = time_perm_oracle(M, args.cpu_seconds)
+    gt.release()
     if world > 1:
-        del g_pool, g_rem, g_warm_rem
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)

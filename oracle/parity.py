@@ -1,4 +1,5 @@
-"""Element-by-element comparison of the CUDA routing outputs with the oracle.
+"""Element-by-element comparison of the CUDA routing outputs with the oracle
+(test infrastructure, like the rest of this package).
 
 Rules (the tolerance and near-tie margin are the ones the routing spec fixes;
 all margins are measured by the oracle in double precision):

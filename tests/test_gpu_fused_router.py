@@ -16,7 +16,7 @@ import torch
 import moe_expert_routing_token_b200 as moe
 import oracle
 from moe_expert_routing_token_b200 import inputs
-from tests import parity
+from oracle import parity
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -105,6 +105,15 @@ def test_workload_full_size(M):
                  renorm=sp.renormalize, G=sp.num_expert_group, TG=sp.topk_group,
                  rsf=sp.routed_scaling_factor)
     assert rep.near_tie <= max(3, len(rows) // 50), rep.summary()
+    # the routing step on every row: the oracle fed the kernel's own logits
+    w_gpu, ids_gpu, logits_gpu = _run(d["hidden"], d["weight"], d["bias"], "ke", sp.topk, sp.renormalize,
+                                      sp.num_expert_group, sp.topk_group, sp.routed_scaling_factor)
+    orc = oracle.biased_grouped_topk(logits_gpu.double().numpy(), d["bias"], sp.topk, sp.renormalize,
+                                     sp.num_expert_group, sp.topk_group, sp.routed_scaling_factor)
+    rep_all = parity.compare(w_gpu.numpy(), ids_gpu.numpy(), orc, E=256, G=sp.num_expert_group,
+                             TG=sp.topk_group, k=sp.topk, renorm=sp.renormalize, rsf=sp.routed_scaling_factor,
+                             fp32_logits=False)
+    assert rep_all.ok() and rep_all.rows == M, "routing of kernel logits, all rows: " + rep_all.summary()
 
 
 def test_without_logits_output_matches():

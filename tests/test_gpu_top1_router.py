@@ -18,7 +18,7 @@ import torch
 import moe_expert_routing_token_b200 as moe
 import oracle
 from moe_expert_routing_token_b200 import inputs
-from tests import parity
+from oracle import parity
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -128,6 +128,28 @@ def test_zero_rows_and_equal_logits():
         assert np.all(ids.numpy()[~zero, 0] == 2)
         assert torch.equal(logits[:, 2], logits[:, 5])
         _check(h, w, layout, 30.0)
+
+
+def test_saturated_softcap_ties():
+    """With c = 1, logits 20 and 25 both cap to exactly 1 (tanh saturates in
+    fp32 and in double), so the capped row has two equal largest values.  The
+    kernel picks on the raw logits (expert 1), the oracle takes the lower
+    index among equal capped values (expert 0): both are in the tie set, the
+    row must count as a near tie and pass, and the weight, which depends only
+    on the capped values, is the same for either choice."""
+    M, K, E = 4, 8, 4
+    h = torch.zeros(M, K)
+    h[:, 0] = 1.0
+    w = torch.zeros(E, K)
+    w[0, 0], w[1, 0], w[2, 0], w[3, 0] = 20.0, 25.0, -3.0, 0.5  # exact in bf16
+    h, w = h.to(torch.bfloat16), w.to(torch.bfloat16)
+    for layout in ("ek", "ke"):
+        rep = _check(h, w, layout, 1.0)
+        assert rep.near_tie == M and rep.clear == 0, rep.summary()
+        wt, ids, _ = _run(h, w, layout, 1.0)
+        assert np.all(np.isin(ids.numpy()[:, 0], [0, 1]))
+        expect = 1.0 / (2.0 + np.exp(np.tanh(-3.0) - 1.0) + np.exp(np.tanh(0.5) - 1.0))
+        assert np.allclose(wt.numpy()[:, 0], expect, rtol=W_RTOL, atol=0)
 
 
 def test_empty_batch():

@@ -4,7 +4,7 @@ import numpy as np
 import torch
 
 import oracle
-from tests import parity
+from oracle import parity
 
 E, G, TG, K = 256, 8, 4, 8
 S = E // G
