@@ -240,10 +240,10 @@ int launch_generic(const RouteArgs& a, cudaStream_t st) {
 // the grid to the octets (R rows per warp) capped at one wave of resident
 // blocks, and launch with programmatic dependent launch (the kernel waits for
 // the previous kernel before it reads any input).
-template <typename TIn, int E, int SCORE, bool BIAS, int MODE, int GS>
+template <typename TIn, int E, int L, int SCORE, bool BIAS, int MODE, int GS>
 int launch_direct(const RouteArgs& a, cudaStream_t st) {
-    auto kern = route_direct_kernel<TIn, E, SCORE, BIAS, MODE, GS>;
-    constexpr size_t smem = direct_smem_bytes<TIn, E>();
+    auto kern = route_direct_kernel<TIn, E, L, SCORE, BIAS, MODE, GS>;
+    constexpr size_t smem = direct_smem_bytes<TIn, E, L>();
     int dev = 0, sms = 0, per_sm = 1;
     int rc = device_and_sms(&dev, &sms);
     if (rc != MOE_OK) return rc;
@@ -259,7 +259,7 @@ int launch_direct(const RouteArgs& a, cudaStream_t st) {
     }
     rc = resident_blocks(dev, kern, kDirectThreads, smem, &per_sm);
     if (rc != MOE_OK) return rc;
-    using Shape = DirectShape<TIn, E>;
+    using Shape = DirectShape<TIn, E, L>;
     constexpr int R = Shape::R;
     const int64_t n_oct = (a.M + R - 1) / R;
     // E = 256: the logits seen as rows of 128 bytes, one box of R token rows
@@ -292,20 +292,34 @@ int launch_direct(const RouteArgs& a, cudaStream_t st) {
     return MOE_OK;
 }
 
+// Batches at least this large route bf16 E = 256 rows with 4 lanes per row
+// (fewer instructions per row); smaller ones with 8 (twice the warps, half
+// the serial work per warp, for latency).
+constexpr int64_t kDirectWideRows = 32768;
+
 // The direct kernel's shapes: E = 256 or 160, topk <= 8, every group kept or
 // 8 groups.  Returns -1 for other shapes.
-template <typename TIn, int E, int SCORE, bool BIAS>
-int try_direct_e(const RouteArgs& a, cudaStream_t st) {
+template <typename TIn, int E, int L, int SCORE, bool BIAS>
+int try_direct_el(const RouteArgs& a, cudaStream_t st) {
     constexpr int GS8 = E / 8;  // experts per group with 8 groups
     if (a.TG == a.G) {
-        if constexpr (SCORE == kSigmoid && BIAS) return launch_direct<TIn, E, SCORE, BIAS, kKeyApprox, 0>(a, st);
-        else return launch_direct<TIn, E, SCORE, BIAS, kKeyRaw, 0>(a, st);
+        if constexpr (SCORE == kSigmoid && BIAS) return launch_direct<TIn, E, L, SCORE, BIAS, kKeyApprox, 0>(a, st);
+        else return launch_direct<TIn, E, L, SCORE, BIAS, kKeyRaw, 0>(a, st);
     }
     if (a.G == 8) {
         constexpr int MODE = SCORE == kSigmoid ? kKeyExact : kKeyRaw;
-        return launch_direct<TIn, E, SCORE, BIAS, MODE, GS8>(a, st);
+        return launch_direct<TIn, E, L, SCORE, BIAS, MODE, GS8>(a, st);
     }
     return -1;
+}
+
+template <typename TIn, int E, int SCORE, bool BIAS>
+int try_direct_e(const RouteArgs& a, cudaStream_t st) {
+    if constexpr (E == 160) return try_direct_el<TIn, E, 4, SCORE, BIAS>(a, st);
+    else if constexpr (sizeof(TIn) == 4) return try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
+    else
+        return a.M >= kDirectWideRows ? try_direct_el<TIn, E, 4, SCORE, BIAS>(a, st)
+                                      : try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
 }
 
 template <typename TIn, int SCORE, bool BIAS>

@@ -20,19 +20,19 @@
 //    register order of every lane's experts is its segment order.
 //  * Threshold.  Each lane scores its C experts (selection keys), takes the
 //    maxima of blocks of 8 experts, and the row's four lanes find tau, the
-//    k-th largest block maximum, with a merge network over xor-shuffles: tau
-//    is a lower bound for the k-th best key, since the maxima belong to
-//    distinct experts.  With group selection the kept groups are ranked first
+//    k-th largest of each lane's four largest block maxima, with a merge
+//    network over xor-shuffles: tau is a lower bound for the k-th best key,
+//    since the maxima belong to distinct experts.  With group selection the kept groups are ranked first
 //    and tau is the k-th largest of their top-2 values.
 //  * Candidates.  Experts with key >= tau - band (about 10 per row on the
-//    benchmark workloads) are written, with their exact keys, to a per-row
-//    list; each candidate is then ranked by counting the candidates above it,
-//    and its rank is its output slot, so the ids leave in descending key
-//    order.  Exact keys that tie (bf16 logits repeat, so a few rows per
+//    benchmark workloads) are appended to a per-row list; the row's four
+//    lanes then share the list evenly, compute the exact keys of their
+//    entries and rank each one by counting the candidates above it.  The rank
+//    is the output slot, so the ids leave in descending key order.  Exact keys that tie (bf16 logits repeat, so a few rows per
 //    thousand have them) are detected from the rank sum and ranked again with
 //    ties to the lower expert index.  A row with more than kDirectCap
-//    candidates or fewer than k (massive ties, NaN scores) is routed by k
-//    exact rounds of arg-max.
+//    candidates or fewer than k (massive ties, NaN scores) is routed by the
+//    whole warp: E / 32 exact keys per lane and k rounds of warp arg-max.
 //
 // Selection keys may approximate the exact keys as long as |phase-1 key -
 // exact key| <= eps for every expert: then k experts have exact keys >= tau -
@@ -57,8 +57,6 @@ static __device__ unsigned int g_watchdog_trips_direct;
 
 constexpr int kDirectWarps = 4;
 constexpr int kDirectThreads = kDirectWarps * 32;
-constexpr int kDirectLanes = 4;    // lanes per row
-constexpr int kDirectRows = 8;     // rows per octet (32 / kDirectLanes)
 constexpr int kDirectCap = 32;     // candidates per row on the fast path
 constexpr int kDirectStages = 2;   // octets a warp keeps in flight
 
@@ -101,12 +99,13 @@ constexpr int direct_row_stride(int row_bytes, int seg, int chunks, int epc, int
     return -1;
 }
 
-template <typename TIn, int E>
+// L lanes per row (4 or 8), R = 32 / L rows per warp pass ("octet").
+template <typename TIn, int E, int L_>
 struct DirectShape {
-    static constexpr int L = kDirectLanes;
+    static constexpr int L = L_;
     static constexpr int ESZ = sizeof(TIn);
     static constexpr int C = E / L;                  // experts per lane
-    static constexpr int R = kDirectRows;            // rows per octet
+    static constexpr int R = 32 / L;                 // rows per octet
     static constexpr int ROW_BYTES = E * ESZ;
     static constexpr int SEG = C * ESZ;              // bytes of a lane's segment
     static constexpr int CH = SEG / 16;              // 16-byte chunks per segment
@@ -114,50 +113,50 @@ struct DirectShape {
     static constexpr int CQ = (C / 4) | 1;           // padded bias layout: odd float4 count per lane
     static constexpr int CS = CQ * 4;
     // TMA staging: segments of whole 128-byte swizzle rows
-    static constexpr bool TMA = SEG % 128 == 0;
-    static constexpr int SUB = SEG / 128;            // swizzle rows per segment (TMA)
+    static constexpr bool TMA = E == 256;            // rows of 512 or 1024 bytes: swizzled TMA staging
     static constexpr int TROWS = ROW_BYTES / 128;    // swizzle rows per token row (TMA)
     static constexpr int RS = TMA ? ROW_BYTES : direct_row_stride(ROW_BYTES, SEG, CH, EPC, CS * 4);
     static constexpr int STAGE = R * RS;             // bytes per staged octet (a multiple of 1024 for TMA)
     static constexpr int NB = C / 8;                 // blocks of 8 experts per lane
     static constexpr int MW = (C + 31) / 32;         // candidate mask words per lane
-    static_assert(E % L == 0 && SEG % 16 == 0 && C % 8 == 0 && 8 % EPC == 0, "unsupported direct shape");
+    static_assert((L == 4 || L == 8) && E % L == 0 && SEG % 16 == 0 && C % 8 == 0 && 8 % EPC == 0,
+                  "unsupported direct shape");
     static_assert(RS > 0 && RS % 16 == 0, "no conflict-free staging layout");
     static_assert(!TMA || STAGE % 1024 == 0, "swizzled stages start on 1024-byte boundaries");
     static_assert(MW <= 2, "at most 64 experts per lane");
 };
 
 // Byte offset, within a staged octet, of chunk q (16 bytes) of lane segment s
-// of row r.
-template <typename TIn, int E>
+// of row r.  TMA staging: the 16-byte chunk c of swizzle row sr sits at
+// chunk c ^ (sr mod 8) of that row.
+template <typename S>
 __device__ __forceinline__ int direct_chunk_off(int r, int s, int q) {
-    using S = DirectShape<TIn, E>;
+    const int byte = r * S::ROW_BYTES + s * S::SEG + 16 * q;
     if constexpr (S::TMA) {
-        const int sr = r * S::TROWS + s * S::SUB + q / 8;  // swizzle row
-        return sr * 128 + (((q % 8) ^ (sr & 7)) << 4);
+        const int sr = byte >> 7;
+        return (sr << 7) + ((((byte >> 4) & 7) ^ (sr & 7)) << 4);
     } else {
         return r * S::RS + s * S::SEG + 16 * q;
     }
 }
 
 // Per-warp candidate lists: R rows of up to kDirectCap entries.  key:
-// orderable exact key (0 pads the list), p: the unbiased score (sigmoid) or
-// the logit (softmax), id: the expert.  Row strides are an odd number of
-// 16-byte vectors (key) or of words (p, id), so that the rows of a warp fall
-// in different banks.
+// orderable exact key (0 pads the list), id: the expert; out: the winners by
+// output slot, (p, id) with p the unbiased score (sigmoid) or the logit
+// (softmax).  Row strides are an odd number of 16-byte vectors (key) or of
+// words (id), so that the rows of a warp fall in different banks.
 constexpr int kListKeyStride = kDirectCap + 4;  // 36 words: 9 vectors
 constexpr int kListStride = kDirectCap + 1;     // 33 words
 template <int R>
 struct DirectLists {
     uint32_t key[R][kListKeyStride];
-    float p[R][kListStride];
     int id[R][kListStride];
     float2 out[R][9];  // by output slot: (p, id) of the winner
 };
 
-template <typename TIn, int E>
+template <typename TIn, int E, int L>
 constexpr size_t direct_smem_bytes() {
-    using S = DirectShape<TIn, E>;
+    using S = DirectShape<TIn, E, L>;
     return 1024 + (size_t)kDirectWarps * kDirectStages * S::STAGE +     // staged octets
            (size_t)kDirectWarps * sizeof(DirectLists<S::R>) +          // candidate lists
            (size_t)S::L * S::CS * 4 + (size_t)E * 4 +                  // bias tables
@@ -186,13 +185,13 @@ __device__ __forceinline__ void sort_desc(float (&v)[N]) {
     }
 }
 
-// The K-th largest (1 <= K <= 8) and the largest of the 4 * P values held P
-// per lane by the 4 lanes of a row (P = 4 or 8, any order; -inf pads).  Sort
-// locally, then two xor-shuffle rounds each merge two sorted lists:
+// The K-th largest (1 <= K <= 8) and the largest of the L * P values held P
+// per lane by the L lanes of a row (P = 4 or 8, any order; -inf pads).  Sort
+// locally, then log2(L) xor-shuffle rounds each merge two sorted lists:
 // concatenation while the result fits in 8, else the top 8 of the two
 // (elementwise max against the reversed partner, a bitonic sequence).  For
 // K = 8 the last round needs only the minimum of that top 8.
-template <int P>
+template <int P, int L>
 __device__ __forceinline__ float row_kth(const float (&in)[P], int K, float& vmax) {
     float a[8];
     {
@@ -215,12 +214,14 @@ __device__ __forceinline__ float row_kth(const float (&in)[P], int K, float& vma
         for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], b[7 - i]);
         bitonic_clean_desc(a);
     }
-    {
+#pragma unroll
+    for (int o = 2; o < L; o <<= 1) {
         float b[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = __shfl_xor_sync(kFullMask, a[i], 2);
+        for (int i = 0; i < 8; ++i) b[i] = __shfl_xor_sync(kFullMask, a[i], o);
 #pragma unroll
         for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], b[7 - i]);
+        if ((o << 1) < L) bitonic_clean_desc(a);
     }
     if (K == 8) {
         vmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
@@ -275,10 +276,10 @@ __device__ __forceinline__ void exact_key(float x, float b, float& key, float& p
 
 // GS: experts per group when groups are selected (the lane owns C / GS whole
 // groups), 0 when every group is kept.
-template <typename TIn, int E, int SCORE, bool BIAS, int MODE, int GS>
+template <typename TIn, int E, int L_, int SCORE, bool BIAS, int MODE, int GS>
 __global__ void __launch_bounds__(kDirectThreads)
     route_direct_kernel(const __grid_constant__ CUtensorMap tmap, RouteArgs a, int64_t n_oct) {
-    using S = DirectShape<TIn, E>;
+    using S = DirectShape<TIn, E, L_>;
     constexpr int C = S::C, R = S::R, L = S::L, D = kDirectStages, EPC = S::EPC, CH = S::CH;
     constexpr bool GROUPED = GS > 0;
     constexpr int NG = GROUPED ? C / GS : 1;  // groups per lane
@@ -388,7 +389,7 @@ __global__ void __launch_bounds__(kDirectThreads)
         const uint8_t* stage = my_stages + (size_t)d * S::STAGE;
         // logit of lane-local expert li of segment s_ of this lane's row
         auto logit_at = [&](int s_, int li) {
-            return staged_logit<TIn>(stage + direct_chunk_off<TIn, E>(rr, s_, li / EPC), li % EPC);
+            return staged_logit<TIn>(stage + direct_chunk_off<S>(rr, s_, li / EPC), li % EPC);
         };
         const int64_t row = oct * R + rr;
         const bool valid = row < a.M;
@@ -398,7 +399,7 @@ __global__ void __launch_bounds__(kDirectThreads)
 #pragma unroll
         for (int q = 0; q < CH; ++q) {
             const int c = q;
-            const uint4 v = *reinterpret_cast<const uint4*>(stage + direct_chunk_off<TIn, E>(rr, sl, q));
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + direct_chunk_off<S>(rr, sl, q));
             if constexpr (MODE == kKeyApprox) {
                 float h[EPC];
                 if constexpr (sizeof(TIn) == 2) {
@@ -475,25 +476,44 @@ __global__ void __launch_bounds__(kDirectThreads)
                     for (int u = 0; u < NG; ++u) rank[u] += (o > gsc[u]) || (o == gsc[u] && og < sl * NG + u);
                 }
             }
-            constexpr int TV = (2 * NG <= 4) ? 4 : 8;
-            float tv[TV];
+            static_assert(NG <= 2, "at most two groups per lane");
+            constexpr int BSZ = GS / 4;  // four blocks per group
             float mx = -INFINITY;
 #pragma unroll
             for (int u = 0; u < NG; ++u) mx = fmaxf(mx, m1[u]);
-#pragma unroll
-            for (int i = 0; i < TV; ++i) tv[i] = -INFINITY;
             bool kept[NG];
+            float tv[4];
+            {
+                float bm[8];
 #pragma unroll
-            for (int u = 0; u < NG; ++u) {
-                kept[u] = rank[u] < a.TG;
-                tv[2 * u] = kept[u] ? m1[u] : -INFINITY;
-                tv[2 * u + 1] = kept[u] ? m2[u] : -INFINITY;
+                for (int u = 0; u < NG; ++u) {
+                    kept[u] = rank[u] < a.TG;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        float m = -INFINITY;
+#pragma unroll
+                        for (int i = 0; i < BSZ; ++i) m = fmaxf(m, key[u * GS + b * BSZ + i]);
+                        bm[4 * u + b] = kept[u] ? m : -INFINITY;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tv[i] = bm[i];
+                if constexpr (NG == 2) {
+                    float h[4] = {bm[4], bm[5], bm[6], bm[7]};
+                    sort_desc(tv);
+                    sort_desc(h);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) tv[i] = fmaxf(tv[i], h[3 - i]);
+                }
             }
+            // experts of dropped groups are not admissible
 #pragma unroll
             for (int i = 0; i < C; ++i)
                 if (!kept[i / GS]) keep_bits[i / 32] &= ~(1u << (i % 32));
+            // the k-th largest of the kept groups' block maxima (distinct
+            // experts: a lower bound for the k-th best admissible key)
             float dummy;
-            tau = row_kth<TV>(tv, K, dummy);
+            tau = row_kth<4, L>(tv, K, dummy);
             rowmax = mx;
 #pragma unroll
             for (int o = 1; o < L; o <<= 1) rowmax = fmaxf(rowmax, __shfl_xor_sync(kFullMask, rowmax, o));
@@ -506,12 +526,18 @@ __global__ void __launch_bounds__(kDirectThreads)
                 const float* k8 = key + 8 * u;
                 bm[u] = fmax3(fmax3(k8[0], k8[1], k8[2]), fmax3(k8[3], k8[4], k8[5]), fmaxf(k8[6], k8[7]));
             }
-            if constexpr (S::NB <= 4) {
-                float b4[4] = {bm[0], bm[1], bm[2], bm[3]};
-                tau = row_kth<4>(b4, K, rowmax);
-            } else {
-                tau = row_kth<8>(bm, K, rowmax);
+            // Each lane contributes its four largest block maxima (the 16 of
+            // the row are distinct experts, so their k-th largest is still a
+            // lower bound): two sorted halves, then the top four of the two.
+            float b4[4] = {bm[0], bm[1], bm[2], bm[3]};
+            if constexpr (S::NB > 4) {
+                float h[4] = {bm[4], bm[5], bm[6], bm[7]};
+                sort_desc(b4);
+                sort_desc(h);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) b4[i] = fmaxf(b4[i], h[3 - i]);
             }
+            tau = row_kth<4, L>(b4, K, rowmax);
         }
         const float lo = tau - band;
 
@@ -545,7 +571,10 @@ __global__ void __launch_bounds__(kDirectThreads)
         const int n = __shfl_sync(kFullMask, incl, seg0 + L - 1);
         bool slow = valid && (n > kDirectCap || n < K);
 
-        // ---- exact keys of the candidates -----------------------------------
+        // ---- candidate list: ids first, then exact keys by list position ----
+        // Each lane appends its candidates' ids; then the row's four lanes take
+        // the list entries t = sl, sl + 4, ... (an even share, whatever lane the
+        // experts live in), compute their exact keys and rank them.
         if (!slow) {
             int pos = incl - cnt;
 #pragma unroll
@@ -554,38 +583,64 @@ __global__ void __launch_bounds__(kDirectThreads)
                 while (bits) {
                     const int i = w * 32 + __ffs(bits) - 1;
                     bits &= bits - 1u;
-                    const int e = sl * C + i;
-                    float kx, px;
-                    exact_key<SCORE, BIAS, MODE>(logit_at(sl, i), BIAS ? s_b2[e] : 0.0f, kx, px);
-                    lst.key[rr][pos] = order_u32(kx);
-                    lst.p[rr][pos] = px;
-                    lst.id[rr][pos] = e;
-                    ++pos;
+                    lst.id[rr][pos++] = sl * C + i;
                 }
             }
         }
         const int nf = (valid && !slow) ? n : 0;
         const int nmax = __reduce_max_sync(kFullMask, nf);
         const int jmax = (nmax + 3) & ~3;
-        for (int u = nf + sl; u < jmax; u += L) lst.key[rr][u] = 0u;
+        __syncwarp();
+        constexpr int TPL = kDirectCap / L;  // list entries per lane
+        uint32_t kt[TPL];
+        float pt[TPL];
+        int it[TPL];
+#pragma unroll
+        for (int u = 0; u < TPL; ++u) {
+            const int t = sl + u * L;
+            kt[u] = 0u;
+            pt[u] = 0.0f;
+            it[u] = 0;
+            if (u * L < nmax) {  // warp-uniform bound
+                if (t < nf) {
+                    const int e = lst.id[rr][t];
+                    float kx, px;
+                    exact_key<SCORE, BIAS, MODE>(logit_at(e / C, e % C), BIAS ? s_b2[e] : 0.0f, kx, px);
+                    kt[u] = order_u32(kx);
+                    pt[u] = px;
+                    it[u] = e;
+                }
+                if (t < jmax) lst.key[rr][t] = kt[u];  // 0 pads the list to jmax
+            }
+        }
         __syncwarp();
 
         // ---- rank by counting: slot of candidate t = #candidates above it ---
-        // The winners (rank < K) go to the row's slot table.
+        // set.gt gives -1 per key above; three-input adds sum them.  The
+        // winners (rank < K) go to the row's slot table.
         int rsum = 0;
 #pragma unroll
-        for (int u = 0; u < (kDirectCap + L - 1) / L; ++u) {
+        for (int u = 0; u < TPL; ++u) {
             if (u * L < nmax) {  // warp-uniform bound
                 const int t = sl + u * L;
-                const uint32_t kt = t < nf ? lst.key[rr][t] : 0xffffffffu;
+                const uint32_t k0 = t < nf ? kt[u] : 0xffffffffu;
                 int c = 0;
-                for (int j4 = 0; j4 < jmax; j4 += 4) {
-                    const uint4 k4 = *reinterpret_cast<const uint4*>(&lst.key[rr][j4]);
-                    c += (k4.x > kt) + (k4.y > kt) + (k4.z > kt) + (k4.w > kt);
+#pragma unroll
+                for (int j4 = 0; j4 < kDirectCap; j4 += 4) {
+                    if (j4 < jmax) {
+                        const uint4 k4 = *reinterpret_cast<const uint4*>(&lst.key[rr][j4]);
+                        uint32_t s0, s1, s2, s3;
+                        asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s0) : "r"(k4.x), "r"(k0));
+                        asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s1) : "r"(k4.y), "r"(k0));
+                        asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s2) : "r"(k4.z), "r"(k0));
+                        asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s3) : "r"(k4.w), "r"(k0));
+                        c = c - (int)s0 - (int)s1;
+                        c = c - (int)s2 - (int)s3;
+                    }
                 }
                 if (t < nf) {
                     rsum += c;
-                    if (c < K) lst.out[rr][c] = make_float2(lst.p[rr][t], __int_as_float(lst.id[rr][t]));
+                    if (c < K) lst.out[rr][c] = make_float2(pt[u], __int_as_float(it[u]));
                 }
             }
         }
@@ -597,56 +652,82 @@ __global__ void __launch_bounds__(kDirectThreads)
         const bool ties = valid && !slow && rsum != n * (n - 1) / 2;
         if (__any_sync(kFullMask, ties)) {
             __syncwarp();  // the first ranking's slot writes land before these
-#pragma unroll 1
-            for (int t = sl; t < nmax; t += L) {
-                const uint32_t kt = t < nf ? lst.key[rr][t] : 0xffffffffu;
-                const int it = t < nf ? lst.id[rr][t] : 0;
-                int c = 0;
-                for (int jj = 0; jj < nf; ++jj) {
-                    const uint32_t kj = lst.key[rr][jj];
-                    c += (kj > kt) || (kj == kt && lst.id[rr][jj] < it);
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) {
+                const int t = sl + u * L;
+                if (u * L < nmax) {
+                    int c = 0;
+                    for (int jj = 0; jj < nf; ++jj) {
+                        const uint32_t kj = lst.key[rr][jj];
+                        c += (kj > kt[u]) || (kj == kt[u] && lst.id[rr][jj] < it[u]);
+                    }
+                    if (ties && t < nf && c < K) lst.out[rr][c] = make_float2(pt[u], __int_as_float(it[u]));
                 }
-                if (ties && t < nf && c < K) lst.out[rr][c] = make_float2(lst.p[rr][t], __int_as_float(it));
             }
         }
 
-        // ---- rare rows: k exact rounds of arg-max, ties to the lower index ---
-        if (__any_sync(kFullMask, slow)) {
+        // ---- rare rows: the whole warp routes each one by k exact rounds of
+        // arg-max (E / 32 experts per lane), ties to the lower index ----------
+        const unsigned slow_rows = __ballot_sync(kFullMask, slow && sl == 0);
+        if (slow_rows) {
             __syncwarp();
-            const uint64_t keep64 =
-                (uint64_t)keep_bits[0] | (S::MW > 1 ? (uint64_t)keep_bits[S::MW - 1] << 32 : 0ull);
-            uint64_t taken = 0ull;
-#pragma unroll 1
-            for (int jr = 0; jr < K; ++jr) {
-                uint32_t bk = 0u;
-                int bi = 0;
-#pragma unroll 4
-                for (int li = 0; li < C; ++li) {  // ascending index: ties keep the lower index
-                    const int e = sl * C + li;
-                    float kx, px;
-                    exact_key<SCORE, BIAS, MODE>(logit_at(sl, li), BIAS ? s_b2[e] : 0.0f, kx, px);
-                    const bool adm = (((keep64 & ~taken) >> li) & 1ull) != 0ull;
-                    const uint32_t ku = adm ? order_u32(kx) : 0u;
-                    const bool better = ku > bk;
-                    bk = better ? ku : bk;
-                    bi = better ? li : bi;
-                }
-                int be = bk ? sl * C + bi : 0x7fffffff;
+            constexpr int EPL = E / 32;  // experts per lane
+            uint32_t kept_groups = 0xffffffffu;  // of this lane's row, bit g = group g kept
+            if constexpr (GROUPED) {
+                uint32_t own = 0u;
 #pragma unroll
-                for (int o = 1; o < L; o <<= 1) {
-                    const uint32_t ok = __shfl_xor_sync(kFullMask, bk, o);
-                    const int oe = __shfl_xor_sync(kFullMask, be, o);
-                    if (ok > bk || (ok == bk && oe < be)) {
-                        bk = ok;
-                        be = oe;
-                    }
-                }
-                if (be >= sl * C && be < sl * C + C) taken |= 1ull << (be - sl * C);
-                if (slow && sl == 0) {
-                    const int eo = (be >= 0 && be < E) ? be : 0;
+                for (int u = 0; u < NG; ++u) own |= (keep_bits[(u * GS) / 32] >> ((u * GS) % 32) & 1u) << (sl * NG + u);
+#pragma unroll
+                for (int o = 1; o < L; o <<= 1) own |= __shfl_xor_sync(kFullMask, own, o);
+                kept_groups = own;
+            }
+            unsigned left = slow_rows;
+            while (left) {
+                const int src = __ffs(left) - 1;
+                left &= left - 1u;
+                const int r = src / L;
+                const uint32_t km = __shfl_sync(kFullMask, kept_groups, src);
+                auto logit_re = [&](int e) {
+                    const int li = e % C;
+                    return staged_logit<TIn>(stage + direct_chunk_off<S>(r, e / C, li / EPC), li % EPC);
+                };
+                uint32_t ku[EPL];
+#pragma unroll
+                for (int j = 0; j < EPL; ++j) {
+                    const int e = lane * EPL + j;
                     float kx, px;
-                    exact_key<SCORE, BIAS, MODE>(logit_at(eo / C, eo % C), 0.0f, kx, px);
-                    lst.out[rr][jr] = make_float2(px, __int_as_float(eo));
+                    exact_key<SCORE, BIAS, MODE>(logit_re(e), BIAS ? s_b2[e] : 0.0f, kx, px);
+                    const bool adm = GROUPED ? ((km >> (e / (GROUPED ? GS : 1))) & 1u) != 0u : true;
+                    ku[j] = adm ? order_u32(kx) : 0u;
+                }
+#pragma unroll 1
+                for (int jr = 0; jr < K; ++jr) {
+                    uint32_t bk = 0u;
+                    int be = 0x7fffffff;
+#pragma unroll
+                    for (int j = 0; j < EPL; ++j) {
+                        const bool better = ku[j] > bk;  // ascending index: ties keep the lower
+                        be = better ? lane * EPL + j : be;
+                        bk = better ? ku[j] : bk;
+                    }
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) {
+                        const uint32_t ok = __shfl_xor_sync(kFullMask, bk, o);
+                        const int oe = __shfl_xor_sync(kFullMask, be, o);
+                        if (ok > bk || (ok == bk && oe < be)) {
+                            bk = ok;
+                            be = oe;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < EPL; ++j)
+                        if (lane * EPL + j == be) ku[j] = 0u;
+                    if (lane == 0) {
+                        const int eo = (be >= 0 && be < E) ? be : 0;
+                        float kx, px;
+                        exact_key<SCORE, BIAS, MODE>(logit_re(eo), 0.0f, kx, px);
+                        lst.out[r][jr] = make_float2(px, __int_as_float(eo));
+                    }
                 }
             }
         }
