@@ -61,7 +61,7 @@ ROUTING = ("sigmoid", "biased", "grouped", "softmax")
 # Every size the routing spec quotes (the workload, M): the per-config table.
 PER_CONFIG = [("softmax", 64), ("sigmoid", 1), ("sigmoid", 16), ("sigmoid", 64), ("sigmoid", 256),
               ("sigmoid", 4096), ("sigmoid", 16384), ("biased", 4096), ("biased", 32), ("grouped", 16384),
-              ("fused", 8192), ("fused", 64), ("top1", 8192)]
+              ("fused", 8192), ("fused", 64), ("top1", 8192), ("top1", 64)]
 # GPU sleep queued before the start event: about 100 us at the B200's clocks,
 # longer than the host needs to submit the first graph of the timed region.
 SLEEP_CYCLES = 200_000

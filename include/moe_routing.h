@@ -61,8 +61,12 @@ extern "C" {
  * (every version-1 call keeps its signature and meaning).  3: adds the
  * small-E top-1 router moe_fused_router_top1 (earlier calls unchanged).  4:
  * adds moe_fill_shared_expert_slot_philox, the shared-expert slot with the
- * library drawing the shared expert from a seed (earlier calls unchanged). */
-#define MOE_ROUTING_ABI_VERSION 4
+ * library drawing the shared expert from a seed (earlier calls unchanged).
+ * 5: moe_fused_router_top1 takes E up to 256 (its tensor-core kernel);
+ * calls that version 4 accepted still succeed; with (E, K) weights and
+ * K % 64 == 0 they run on the tensor-core kernel, whose fp32 sums are
+ * ordered differently. */
+#define MOE_ROUTING_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -192,18 +196,20 @@ MOE_API int moe_biased_grouped_topk_aiter(const void* gating_output, int dtype, 
 /*
  * moe_fused_router_workspace_size - bytes of device workspace that
  * moe_fused_router_topk needs for these sizes (0 when it needs none).  Small
- * batches (M <= 128) with a long hidden size spread K over several
- * thread-block clusters whose fp32 partial sums meet in the workspace
- * ((clusters x M x 256) floats plus 256 bytes of arrival counters).
- * Returns (size_t)-1 for arguments moe_fused_router_topk would reject.
+ * batches (M <= 128) with a long hidden size (K >= 1024) spread K over up to
+ * 256 CTAs whose fp32 partial logits meet in the workspace: (splits x M x
+ * 256) floats, at most 2 MiB.  Returns (size_t)-1 for arguments
+ * moe_fused_router_topk would reject.
  */
 MOE_API size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E);
 
 /*
  * moe_fused_router_topk - [R] §5 (FusedMoeRouter) with the [R] §4 routing:
  * logits = hidden_states x router_weight accumulated in fp32 on the tensor
- * cores and kept on chip, then the moe_biased_grouped_topk routing of those
- * logits.  The logits never reach device memory unless logits_out is given.
+ * cores, then the moe_biased_grouped_topk routing of those logits.  From
+ * M > 128 (or K < 1024) the logits stay on chip unless logits_out is given;
+ * smaller batches with a long K pass fp32 partial logits through the
+ * workspace to a second launch that sums and routes them.
  *
  *   hidden_states   device, (M, K) bf16
  *   router_weight   device, bf16, (K, E) if weight_layout == MOE_WEIGHT_K_BY_E
@@ -217,11 +223,9 @@ MOE_API size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E);
  *   workspace       device scratch of at least
  *                   moe_fused_router_workspace_size(M, K, E) bytes, 256-byte
  *                   aligned (NULL allowed when that size is 0; otherwise a
- *                   missing or short workspace is MOE_ERR_INVALID_ARG).  It
- *                   must be zero-filled before its first use (its arrival
- *                   counters start at zero); every call leaves it in that
- *                   state again.  Calls that may overlap on the GPU must not
- *                   share one workspace.
+ *                   missing or short workspace is MOE_ERR_INVALID_ARG).  No
+ *                   initial contents are needed.  Calls that may overlap on
+ *                   the GPU must not share one workspace.
  *   other arguments as moe_biased_grouped_topk
  */
 MOE_API int moe_fused_router_topk(const void* hidden_states, const void* router_weight,
@@ -248,16 +252,13 @@ MOE_API int moe_fused_router_topk(const void* hidden_states, const void* router_
  *
  *   Arguments, layouts and results are those of moe_fused_router_topk,
  *   without `workspace` / `workspace_bytes`.
- *   Limit: sizes whose workspace would exceed 2 MiB are rejected with
- *   MOE_ERR_UNSUPPORTED and a message naming the sizes.  With K = 7168 every
- *   M fits (at most 1.75 MiB); K >= 9216 with M close to 128 does not.
- *   Batches above 128 tokens need no scratch and always work.
+ *   Limit: none beyond moe_fused_router_topk's: the workspace of every size
+ *   fits the array (moe_fused_router_workspace_size caps the partial logits
+ *   at 2 MiB).  Batches above 128 tokens need no scratch.
  *   Memory: nothing is allocated or freed.  Every GPU that loads the library
  *   keeps the 2 MiB array for the life of the process.  The first call on
  *   each device looks up the array's device address (cudaGetSymbolAddress);
  *   make that first call before capturing the stream into a CUDA graph.
- *   Each call clears the array's 256 bytes of arrival counters on `stream`
- *   (cudaMemsetAsync) before launching.
  *   Concurrency: all calls on a device share the one array, which keeps the
  *   last call's partial sums; calls that overlap on the GPU (different
  *   streams, or host threads racing on one device) race on it and give wrong
@@ -272,30 +273,32 @@ MOE_API int moe_fused_router_topk_noalloc(const void* hidden_states, const void*
                                           int32_t* topk_ids, float* logits_out, void* stream);
 
 /*
- * moe_fused_router_top1 - the CUDA-core fused router of [R] §5 for small
- * expert counts: per token row,
+ * moe_fused_router_top1 - the fused top-1 router of [R] §5: per token row,
  *     l_e = sum_k h[k] * W(k, e)              (bf16 inputs, fp32 sums)
  *     id  = arg-max_e l_e                     (lower index among equal logits)
  *     w   = 1 / sum_e exp(cap(l_e) - cap(l_id)),  cap(x) = softcap * tanh(x / softcap)
  * i.e. softcapping (when softcap != 0; 0 = none), then top-1 with the
  * softmax probability of the chosen expert as its weight (the page's
- * invsumexp).  cap is strictly increasing, so the arg-max of the raw logits
- * is the arg-max of the capped ones.
+ * invsumexp).  cap is increasing, so the arg-max of the raw logits is an
+ * arg-max of the capped ones.
  *
  *   hidden_states   device, (M, K) bf16, 16-byte aligned
  *   router_weight   device, bf16, (K, E) if weight_layout == MOE_WEIGHT_K_BY_E
  *                   or (E, K) if MOE_WEIGHT_E_BY_K (the page's layout),
  *                   16-byte aligned
- *   K               hidden size, a positive multiple of 8
- *   E               experts, 1..8 (else MOE_ERR_UNSUPPORTED); the page sends
- *                   E > 8 to its tensor-core kernel
+ *   K               hidden size, a positive multiple of 8 (of 64 for E > 8)
+ *   E               experts, 1..256 (see the dispatch below)
  *   softcap         finite; 0 = no softcapping; c and -c give the same result
  *   topk_weights    device, (M, 1) fp32 out
- *   topk_ids        device, (M, 1) int32 out
+ *   topk_ids        device, (M, 1) int32 out; -1 only if a kernel wait timed
+ *                   out (moe_watchdog_trips counts it)
  *   logits_out      device, (M, E) fp32 out, or NULL (debug: the raw logits)
- * Every batch size runs on the CUDA cores: at E <= 8 the projection does at
- * most 8 flops per byte of hidden state, below the fp32 CUDA-core ridge (the
- * page's batch-size switch to tensor cores has no counterpart here).
+ * Dispatch: the tensor-core kernel (tcgen05, TMEM accumulator) when
+ * K % 64 == 0, the layout is (E, K) and E <= 256, at every batch size (the
+ * page switches to tensor cores from 512 tokens or E > 8; below that the
+ * tensor-core kernel measured faster here too); otherwise the CUDA-core
+ * kernel, which takes E <= 8 and K % 8 == 0.  E > 8 outside the tensor-core
+ * conditions is MOE_ERR_UNSUPPORTED.
  * Asynchronous on `stream`; no allocation; M == 0 launches nothing.
  */
 MOE_API int moe_fused_router_top1(const void* hidden_states, const void* router_weight, int weight_layout,

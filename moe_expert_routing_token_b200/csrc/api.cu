@@ -21,6 +21,7 @@
 #include "routing_kernels.cuh"
 #include "routing_staged.cuh"
 #include "routing_stream.cuh"
+#include "routing_warp.cuh"
 #include "tma_host.cuh"
 
 namespace moe {
@@ -292,6 +293,56 @@ int launch_direct(const RouteArgs& a, cudaStream_t st) {
     return MOE_OK;
 }
 
+// Batches up to this size route one row per warp (route_warp_kernel): the
+// shortest chain per row.  Measured on B200 (bf16 E = 256, k = 8): 2.3 us at
+// M = 64 and 5.1 us at M = 4096 (direct kernel: 4.3 and 5.8 us); from
+// M = 8192 the direct kernel's fewer instructions per row win (5.9 against
+// 8.2 us).
+constexpr int64_t kWarpRowMaxRows = 4096;
+
+template <typename TIn, int E, int SCORE, bool BIAS, bool GROUPED>
+int launch_warp_rows(const RouteArgs& a, cudaStream_t st) {
+    auto kern = route_warp_kernel<TIn, E, SCORE, BIAS, GROUPED>;
+    int dev = 0, sms = 0;
+    int rc = device_and_sms(&dev, &sms);
+    if (rc != MOE_OK) return rc;
+    const int64_t need = (a.M + kWarpRowWarps - 1) / kWarpRowWarps;
+    const int64_t cap = (int64_t)sms * 16;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(need < cap ? need : cap), 1, 1);
+    cfg.blockDim = dim3((unsigned)kWarpRowThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kern, a);
+    if (err != cudaSuccess) return cuda_fail(err, "warp-per-row routing kernel launch");
+    return MOE_OK;
+}
+
+// The warp-per-row kernel's shapes: E = 256 or 160 (C = E / 32 experts per
+// lane), groups of whole lanes (G divides 32), decode-sized batches; 16-byte
+// aligned rows where a lane's segment is read with 16-byte loads.  Returns -1
+// otherwise.
+template <typename TIn, int E, int SCORE, bool BIAS>
+int try_warp_rows_e(const RouteArgs& a, cudaStream_t st) {
+    constexpr int SEGB = (E / 32) * (int)sizeof(TIn);
+    if (SEGB % 16 == 0 && !aligned(a.logits, 16)) return -1;
+    if (a.G > 1 && a.TG < a.G) return launch_warp_rows<TIn, E, SCORE, BIAS, true>(a, st);
+    return launch_warp_rows<TIn, E, SCORE, BIAS, false>(a, st);
+}
+
+template <typename TIn, int SCORE, bool BIAS>
+int try_warp_rows(const RouteArgs& a, cudaStream_t st) {
+    if (a.M > kWarpRowMaxRows || 32 % a.G != 0) return -1;
+    if (a.E == 256) return try_warp_rows_e<TIn, 256, SCORE, BIAS>(a, st);
+    if (a.E == 160) return try_warp_rows_e<TIn, 160, SCORE, BIAS>(a, st);
+    return -1;
+}
+
 // Batches at least this large route bf16 E = 256 rows with 4 lanes per row
 // (fewer instructions per row); smaller ones with 8 (twice the warps, half
 // the serial work per warp, for latency).
@@ -315,8 +366,7 @@ int try_direct_el(const RouteArgs& a, cudaStream_t st) {
 
 template <typename TIn, int E, int SCORE, bool BIAS>
 int try_direct_e(const RouteArgs& a, cudaStream_t st) {
-    if constexpr (E == 160) return try_direct_el<TIn, E, 4, SCORE, BIAS>(a, st);
-    else if constexpr (sizeof(TIn) == 4) return try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
+    if constexpr (sizeof(TIn) == 4) return try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
     else
         return a.M >= kDirectWideRows ? try_direct_el<TIn, E, 4, SCORE, BIAS>(a, st)
                                       : try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
@@ -327,14 +377,20 @@ int try_direct(const RouteArgs& a, cudaStream_t st) {
     if (a.K > 8 || !aligned(a.logits, 16)) return -1;
     // TMA box coordinates are 32-bit: (M * 8) rows of 128 bytes at most
     if (a.M > (int64_t(1) << 28)) return -1;
+    // E = 160 (rows staged by per-row copies) measured slower than the
+    // two-phase streaming kernel at every size it would serve (fp32, k = 6,
+    // G = 8: 15.8 against 9.7 us at M = 16384), so it is left to that kernel.
     if (a.E == 256) return try_direct_e<TIn, 256, SCORE, BIAS>(a, st);
-    if (a.E == 160) return try_direct_e<TIn, 160, SCORE, BIAS>(a, st);
     return -1;
 }
 
 template <typename TIn, int SCORE, bool BIAS>
 int dispatch_typed(const RouteArgs& a, cudaStream_t st) {
     const int E = a.E;
+    {
+        const int rc = try_warp_rows<TIn, SCORE, BIAS>(a, st);
+        if (rc >= 0) return rc;
+    }
     {
         const int rc = try_direct<TIn, SCORE, BIAS>(a, st);
         if (rc >= 0) return rc;
@@ -452,7 +508,12 @@ int moe_watchdog_trips(unsigned int* count) {
     if (rc != MOE_OK) return rc;
     rc = moe::read_fused_watchdog(&b);
     if (rc != MOE_OK) return rc;
-    *count = a + b;
+    unsigned int c = 0, d = 0;
+    rc = moe::read_top1_watchdog(&c);
+    if (rc != MOE_OK) return rc;
+    rc = moe::read_decode_watchdog(&d);
+    if (rc != MOE_OK) return rc;
+    *count = a + b + c + d;
     return MOE_OK;
 }
 

@@ -16,10 +16,11 @@
 //               distributed shared memory (each CTA of the cluster owns
 //               128/SPLIT rows and receives the other CTAs' partials for
 //               them), summed in a fixed rank order, staged in shared memory
-//               and routed by the same SegRouter body as the routing kernels.
+//               and routed one row per warp by the warp-per-row routing body.
 // The K dimension is split across the SPLIT CTAs of a cluster so that enough
-// SMs stream the hidden states (M=8192: 64 tiles x 2 = 128 CTAs; decode
-// M=64: 1 tile x 16).  Every barrier wait is bounded.
+// SMs stream the hidden states (M=8192: 64 tiles x 2 = 128 CTAs).  A single
+// tile with a long K (decode batches, M <= 128) takes fused_decode.cu
+// instead.  Every barrier wait is bounded.
 #include <cstdio>
 #include <mutex>
 #include <type_traits>
@@ -28,6 +29,7 @@
 #include "fused_router.cuh"
 #include "moe_routing.h"
 #include "routing_kernels.cuh"
+#include "routing_warp.cuh"
 #include "sm100_ptx.cuh"
 #include "tma_host.cuh"
 
@@ -57,25 +59,11 @@ struct FusedArgs {
     float* logits_out;  // (M, 256) fp32 or nullptr
     int num_kb;         // K / 64
     int kb_per_split;   // k-blocks per CTA
-    int ncl;            // clusters per tile whose partials meet in the workspace (1: none)
-    float* ws_part;     // [ncl][M][256] fp32 cluster partials (ncl > 1)
-    unsigned int* ws_ticket;  // [SPLIT] arrival counters, zero between calls (ncl > 1)
 };
 
-// Workspace of the wide split-K path (one 128-row tile over several clusters).
-constexpr int kWideSplit = 8;     // CTAs per cluster on that path
-constexpr int kWideMaxClusters = 18;
-constexpr int kWideMinKb = 16;    // k-blocks below which one cluster suffices
-
-__host__ __device__ constexpr int wide_clusters(int num_kb) {
-    const int c = (num_kb + kWideSplit - 1) / kWideSplit;
-    return c > kWideMaxClusters ? kWideMaxClusters : c;
-}
-
-size_t wide_workspace_bytes(int64_t M, int num_kb) {
-    const size_t part = (size_t)wide_clusters(num_kb) * (size_t)M * kBN * sizeof(float);
-    return (part + 255) / 256 * 256 + 256;
-}
+// One 128-row tile with at least this many k-blocks takes the decode path
+// (fused_decode.cu): K split over CTAs, partial logits in the workspace.
+constexpr int kDecodeMinKb = 16;
 
 // Bytes at the start of shared memory used first as the stage ring, then (after
 // the main loop) as the split-K exchange and routing area.  With SPLIT = 2 that
@@ -94,21 +82,7 @@ __host__ __device__ constexpr size_t fused_smem_bytes() {
     return 1024 + kOverlayBytes + Router::BIAS_FLOATS * 4 + 256;
 }
 
-// Owner-side staged logits row: chunk c (32 floats) at c * 36.
-__device__ __forceinline__ int fin_off(int r, int col) { return r * kFinStride + (col >> 5) * 36 + (col & 31); }
-
-template <int SPLIT>
-struct FinScores {
-    const float* fin;
-    int warp_row0;
-    __device__ __forceinline__ void store(int, float, float, float, float) const {}
-    __device__ __forceinline__ float get(int seg, int e) const {
-        const int r = warp_row0 + seg;  // rows past the owned range are padding
-        return r < kBM / SPLIT ? sigmoid_f32(fin[fin_off(r, e)]) : 0.0f;
-    }
-};
-
-template <int SPLIT, bool B_MN_MAJOR, bool BIAS, bool GRED>
+template <int SPLIT, bool B_MN_MAJOR, bool BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_router_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         FusedArgs fa) {
@@ -126,7 +100,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 3);
     volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* s_peer_abort = s_abort + 1;
-    volatile int* s_last = s_abort + 2;  // this CTA reduces the clusters' partials
     // Overlays of the stage ring, valid once the main loop is over: one slot
     // of partial sums per source CTA for the rows this CTA owns, in the
     // chunked staged-row layout; slot 0 is summed in place and then holds
@@ -143,9 +116,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = ptx::cluster_ctarank();
-    const int cl = GRED ? (int)((blockIdx.x / SPLIT) % fa.ncl) : 0;   // cluster within the tile
-    const int m_tile = GRED ? (int)(blockIdx.x / (SPLIT * fa.ncl)) : (int)(blockIdx.x / SPLIT);
-    const int kb0 = (cl * SPLIT + (int)rank) * fa.kb_per_split;
+    const int m_tile = (int)(blockIdx.x / SPLIT);
+    const int kb0 = (int)rank * fa.kb_per_split;
     int nkb = fa.num_kb - kb0;
     if (nkb > fa.kb_per_split) nkb = fa.kb_per_split;
     if (nkb < 0) nkb = 0;
@@ -161,7 +133,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(sent_bar, 1);
         *s_abort = 0;
         *s_peer_abort = 0;
-        *s_last = 1;
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
@@ -264,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_acc = nkb > 0;           // uniform over the CTA
     float* const recv = slots + (size_t)ROWS * kFinStride;  // SPLIT = 2: partner's partials [ROWS][260]
     float* const send = recv + (size_t)ROWS * kPairStride;  // SPLIT = 2: rows the partner owns [ROWS][260]
-    if constexpr (SPLIT == 2 && !GRED) {
+    if constexpr (SPLIT == 2) {
         // Own rows go to the staged layout, the partner's rows to a compact
         // send buffer that one bulk copy moves into the partner's receive
         // area (16-byte stores across the cluster are far slower).
@@ -354,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*s_abort && part == 0)
             ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(const_cast<int*>(s_peer_abort)), owner), 1u);
     }
-    if constexpr (SPLIT != 2 || GRED) ptx::cluster_sync();
+    if constexpr (SPLIT != 2) ptx::cluster_sync();
 
     // Sum the SPLIT partials of the owned rows in rank order, all 128
     // epilogue threads in parallel, in place into slot 0.
@@ -373,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             float4 acc = *reinterpret_cast<const float4*>(slots + off);
-            if constexpr (SPLIT == 2 && !GRED) {
+            if constexpr (SPLIT == 2) {
                 // two partials: the sum is the same in either order
                 const float4 v = *reinterpret_cast<const float4*>(recv + (size_t)lr * kPairStride + col);
                 acc.x += v.x;
@@ -391,64 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             *reinterpret_cast<float4*>(slots + off) = acc;
-            if (!GRED && fa.logits_out != nullptr && grow < fa.route.M)
+            if (fa.logits_out != nullptr && grow < fa.route.M)
                 *reinterpret_cast<float4*>(fa.logits_out + grow * kBN + col) = acc;
         }
     }
-    if constexpr (GRED) {
-        // Across clusters: publish this cluster's partial of the owned rows;
-        // the last cluster to arrive sums all of them in cluster order.
-        if (epi) {
-            constexpr int COLS = kBN * ROWS / (kEpiWarps * 32);
-            const int t = threadIdx.x - 64;
-            const int lr = t % ROWS;
-            const int col0 = (t / ROWS) * COLS;
-            const int64_t grow = row_base + lr;
-            if (grow < fa.route.M) {
-                float* dst = fa.ws_part + ((size_t)cl * fa.route.M + grow) * kBN;
-                for (int col = col0; col < col0 + COLS; col += 4)
-                    *reinterpret_cast<float4*>(dst + col) =
-                        *reinterpret_cast<const float4*>(slots + lr * kFinStride + (col >> 5) * 36 + (col & 31));
-            }
-            ptx::named_barrier_sync(1, kEpiWarps * 32);
-            if (t == 0) {
-                __threadfence();  // the block's partial writes, ordered by the barrier, before the ticket
-                *s_last = (atomicAdd(&fa.ws_ticket[rank], 1u) == (unsigned)(fa.ncl - 1)) ? 1 : 0;
-            }
-            ptx::named_barrier_sync(1, kEpiWarps * 32);
-            if (*s_last) {
-                __threadfence();
-                for (int col = col0; col < col0 + COLS; col += 4) {
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (grow < fa.route.M) {
-                        // gather 6 partials at a time, add them in cluster order
-                        for (int g0 = 0; g0 < fa.ncl; g0 += 6) {
-                            float4 part[6];
-#pragma unroll
-                            for (int j = 0; j < 6; ++j)
-                                if (g0 + j < fa.ncl)
-                                    part[j] = __ldcg(reinterpret_cast<const float4*>(
-                                        fa.ws_part + ((size_t)(g0 + j) * fa.route.M + grow) * kBN + col));
-#pragma unroll
-                            for (int j = 0; j < 6; ++j) {
-                                if (g0 + j < fa.ncl) {
-                                    acc.x += part[j].x;
-                                    acc.y += part[j].y;
-                                    acc.z += part[j].z;
-                                    acc.w += part[j].w;
-                                }
-                            }
-                        }
-                        if (fa.logits_out != nullptr)
-                            *reinterpret_cast<float4*>(fa.logits_out + grow * kBN + col) = acc;
-                    }
-                    *reinterpret_cast<float4*>(slots + lr * kFinStride + (col >> 5) * 36 + (col & 31)) = acc;
-                }
-                if (t == 0) fa.ws_ticket[rank] = 0u;  // ready for the next call
-            }
-        }
-    }
-    if constexpr (SPLIT == 2 && !GRED) {
+    if constexpr (SPLIT == 2) {
         // The router scratch overlays the send buffer: wait until the partner
         // confirms our partials arrived.
         if (epi && !ptx::mbar_wait_cluster(sent_bar, 0, kWaitNs)) {
@@ -463,44 +381,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_dealloc(tmem, 256);
     }
 
-    // Routing of the owned rows by the epilogue warps (4 rows each per pass).
-    if (epi && *s_last) {
+    // Routing of the owned rows: one warp per row (the warp-per-row routing
+    // kernel's body), the epilogue warps taking rows ew, ew + 16, ...
+    if (epi) {
         const bool aborted = *s_abort || *s_peer_abort;
         const int ew = warp - 2;
-        const int seg = lane / R_t::L;
-        const int e0 = (lane % R_t::L) * 32;
-        for (int base = 0; base < ROWS; base += kEpiWarps * R_t::R) {
-            const int warp_row0 = base + ew * R_t::R;
-            const int lr = warp_row0 + seg;
+        auto* wscr = reinterpret_cast<WarpRowScratch*>(scratch) + ew;
+        static_assert(kEpiWarps * sizeof(WarpRowScratch) <= kEpiWarps * sizeof(typename R_t::Scratch),
+                      "warp routing scratch");
+        // lane l holds experts [8 l, 8 l + 8): chunk l / 4 of the staged row
+        const int loff = (lane >> 2) * 36 + (lane & 3) * 8;
+        float bl[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) bl[c] = BIAS ? s_bias[(lane >> 2) * Router::CS + (lane & 3) * 8 + c] : 0.0f;
+        const bool grouped = fa.route.G > 1 && fa.route.TG < fa.route.G;
+        for (int lr = ew; lr < ROWS; lr += kEpiWarps) {
             const int64_t grow = row_base + lr;
-            const bool valid = lr < ROWS && grow < fa.route.M;
-            float x[32];
-            if (lr < ROWS) {
-                const float4* p = reinterpret_cast<const float4*>(fin + fin_off(lr, e0));
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 t = p[i];
-                    x[4 * i] = t.x;
-                    x[4 * i + 1] = t.y;
-                    x[4 * i + 2] = t.z;
-                    x[4 * i + 3] = t.w;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = 0.0f;
-            }
-            R_t::route(x, valid, grow, s_bias, scratch[ew], fa.route, FinScores<SPLIT>{fin, warp_row0});
-            if (aborted && valid && (lane % R_t::L) == 0) {
-                for (int t = 0; t < fa.route.K; ++t) fa.route.ids[grow * fa.route.K + t] = -1;
-            }
+            if (grow >= fa.route.M) break;  // rows ascend
+            float x[8];
+            const float4* src = reinterpret_cast<const float4*>(fin + (size_t)lr * kFinStride + loff);
+            const float4 v0 = src[0], v1 = src[1];
+            x[0] = v0.x; x[1] = v0.y; x[2] = v0.z; x[3] = v0.w;
+            x[4] = v1.x; x[5] = v1.y; x[6] = v1.z; x[7] = v1.w;
+            if (grouped)
+                warp_route_row<256, kSigmoid, BIAS, true>(x, bl, grow, fa.route, *wscr);
+            else
+                warp_route_row<256, kSigmoid, BIAS, false>(x, bl, grow, fa.route, *wscr);
+            if (aborted && lane < fa.route.K) fa.route.ids[grow * fa.route.K + lane] = -1;
         }
     }
 }
 
-template <int SPLIT, bool B_MN, bool BIAS, bool GRED = false>
+template <int SPLIT, bool B_MN, bool BIAS>
 int launch_fused(const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs& fa, int m_tiles,
                  cudaStream_t stream) {
-    auto kern = fused_router_kernel<SPLIT, B_MN, BIAS, GRED>;
+    auto kern = fused_router_kernel<SPLIT, B_MN, BIAS>;
     {
         static std::mutex mu;
         static std::unordered_map<int, bool> done;  // device ordinal -> attributes set
@@ -520,7 +435,7 @@ int launch_fused(const CUtensorMap& tmA, const CUtensorMap& tmB, const FusedArgs
         }
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(m_tiles * SPLIT * fa.ncl), 1, 1);
+    cfg.gridDim = dim3((unsigned)(m_tiles * SPLIT), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = fused_smem_bytes();
     cfg.stream = stream;
@@ -557,7 +472,7 @@ int max_schedulable_split(int dev) {
     auto hit = cached.find(dev);
     if (hit != cached.end()) return hit->second;
     int best = 8;
-    auto kern = fused_router_kernel<16, false, true, false>;
+    auto kern = fused_router_kernel<16, false, true>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem_bytes()) ==
             cudaSuccess &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
@@ -626,8 +541,8 @@ size_t moe_fused_router_workspace_size(int64_t M, int32_t K, int32_t E) {
     if (M < 0 || K < 1 || E < 1) return (size_t)-1;
     // A single 128-token tile with a long K spreads K over several clusters
     // whose partial sums meet in the workspace; larger batches need none.
-    if (M >= 1 && M <= moe::kBM && E == 256 && K % 64 == 0 && K / 64 >= moe::kWideMinKb)
-        return moe::wide_workspace_bytes(M, K / 64);
+    if (M >= 1 && M <= moe::kBM && E == 256 && K % 64 == 0 && K / 64 >= moe::kDecodeMinKb)
+        return moe::fused_decode_workspace_bytes(M, K / 64);
     return 0;
 }
 
@@ -736,24 +651,11 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
     fa.logits_out = logits_out;
     fa.num_kb = num_kb;
     fa.kb_per_split = (num_kb + split - 1) / split;
-    fa.ncl = 1;
-    fa.ws_part = nullptr;
-    fa.ws_ticket = nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (ws_need > 0) {
-        // wide split-K: ncl clusters of kWideSplit CTAs, one CTA per SM
-        int ncl = wide_clusters(num_kb);
-        if (ncl > sms / kWideSplit) ncl = sms / kWideSplit;
-        if (ncl < 1) ncl = 1;
-        fa.ncl = ncl;
-        fa.kb_per_split = (num_kb + ncl * kWideSplit - 1) / (ncl * kWideSplit);
-        fa.ws_part = static_cast<float*>(workspace);
-        fa.ws_ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + ws_need - 256);
-        if (b_mn)
-            return correction_bias ? launch_fused<kWideSplit, true, true, true>(tmA, tmB, fa, m_tiles, st)
-                                   : launch_fused<kWideSplit, true, false, true>(tmA, tmB, fa, m_tiles, st);
-        return correction_bias ? launch_fused<kWideSplit, false, true, true>(tmA, tmB, fa, m_tiles, st)
-                               : launch_fused<kWideSplit, false, false, true>(tmA, tmB, fa, m_tiles, st);
+        // one tile with a long K: split K over CTAs whose partial logits meet
+        // in the workspace, then route them (two launches)
+        return launch_fused_decode(tmA, tmB, b_mn, fa.route, logits_out, num_kb, workspace, st);
     }
     if (b_mn)
         return correction_bias ? launch_split<true, true>(split, tmA, tmB, fa, m_tiles, st)
@@ -783,12 +685,6 @@ int moe_fused_router_topk_noalloc(const void* hidden_states, const void* router_
     if (need > 0) {
         int rc = noalloc_scratch(&scratch);
         if (rc != MOE_OK) return rc;
-        // The arrival counters at the end of the scratch must start at zero;
-        // clear them on the call's stream (a previous call that stopped early
-        // could have left them set).
-        cudaError_t err = cudaMemsetAsync(static_cast<char*>(scratch) + need - 256, 0, 256,
-                                          static_cast<cudaStream_t>(stream));
-        if (err != cudaSuccess) return set_cuda_error(err, "cudaMemsetAsync(no-alloc scratch counters)");
     }
     return moe_fused_router_topk(hidden_states, router_weight, weight_layout, correction_bias, M, K, E, topk,
                                  renormalize, num_expert_group, topk_group, routed_scaling_factor, topk_weights,

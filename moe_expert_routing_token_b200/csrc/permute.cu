@@ -9,15 +9,22 @@
 //   ascending within an expert), scatter_indx[i] = the position of pair i,
 //   gate_scal[p] = topk_weights of gather_indx[p].
 //
-// Three passes, deterministic (no atomics decide an order):
-//   1. perm_hist_kernel: one block per tile of kPermTile pairs counts its
-//      experts in shared memory and writes the tile's counts to the workspace.
-//   2. perm_scan_kernel: one block of up to 1024 threads (expert x chunk of
-//      tiles) turns the [tiles][E] counts into expert totals, offsets, and
-//      each tile's first position per expert.
-//   3. perm_scatter_kernel: each warp of a tile takes a contiguous run of the
-//      tile's pairs in order; within a 32-pair piece, lanes holding the same
-//      expert are ranked by __match_any_sync, so pairs keep their index order.
+// Two launches, deterministic (no atomic decides an order):
+//   1. perm_count_kernel: one block per tile of kPermTile pairs counts its
+//      experts in shared memory and writes the tile's counts to the
+//      workspace ([tiles][E] int32).
+//   2. perm_place_kernel (programmatic dependent launch: its set-up overlaps
+//      the first): every block sums, per expert, the counts of the tiles
+//      before its own and of all tiles (coalesced reads of the workspace, which
+//      sits in L2), scans the totals over the experts for the offsets, adds
+//      its warps' counts in warp order, and places its pairs: each warp takes
+//      a contiguous run of the tile's pairs in order; within a 32-pair piece,
+//      lanes holding the same expert are ranked by __match_any_sync, so pairs
+//      keep their index order.  Block 0 writes counts and offsets.
+// With more than kPermPlaceMaxTiles tiles the second step is split in two,
+// so that no block reads every tile's counts: perm_scan_kernel (one block)
+// turns the counts into totals, offsets and each tile's first position per
+// expert, and perm_scatter_kernel places the pairs from those.
 // Ids outside [0, E) are skipped: not counted, scatter_indx = -1.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -37,12 +44,24 @@ constexpr int kPermTile = 1024;    // pairs per block
 constexpr int kPermThreads = 256;  // 8 warps; each warp owns 128 consecutive pairs of the tile
 constexpr int kPermWarps = kPermThreads / 32;
 constexpr int kPermMaxE = 1024;
+// Up to this many tiles every block of the placing launch sums the tile
+// counts itself (tiles x E reads per block, from L2); beyond it a single scan
+// block does (three launches).
+constexpr int kPermPlaceMaxTiles = 512;
 
-__global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* __restrict__ ids, int64_t n, int E,
-                                                                 int32_t* __restrict__ tile_counts) {
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kPermThreads) perm_count_kernel(const int32_t* __restrict__ ids, int64_t n, int E,
+                                                                  int32_t* __restrict__ tile_counts) {
     __shared__ int32_t h[kPermMaxE];
+    griddep_launch_dependents();
     for (int e = threadIdx.x; e < E; e += kPermThreads) h[e] = 0;
     __syncthreads();
+    // the ids may be written by the previous kernel in the stream
+    griddep_wait();
     const int64_t t0 = (int64_t)blockIdx.x * kPermTile;
     for (int j = threadIdx.x; j < kPermTile; j += kPermThreads) {
         const int64_t i = t0 + j;
@@ -53,6 +72,161 @@ __global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* 
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += kPermThreads) tile_counts[(int64_t)blockIdx.x * E + e] = h[e];
+}
+
+__global__ void __launch_bounds__(kPermThreads)
+    perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ weights, int64_t n, int E,
+                      int ntiles, const int32_t* __restrict__ tile_counts, int32_t* __restrict__ counts,
+                      int32_t* __restrict__ offsets, int32_t* __restrict__ gather, int32_t* __restrict__ scatter,
+                      float* __restrict__ gate) {
+    extern __shared__ int32_t wbase[];            // [kPermWarps][E]: next position per (warp, expert)
+    __shared__ int32_t s_wsum[kPermThreads / 32];
+    // [2][ng][E] partial sums of the tile counts (ng * E = 4 * threads), then
+    // s_tot (expert totals, then offsets) and s_pre (pairs in earlier tiles)
+    __shared__ __align__(16) int32_t s_part[2 * kPermMaxE];
+    int32_t* s_tot = s_part;
+    int32_t* s_pre = s_part + kPermMaxE;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kRun = kPermTile / kPermWarps;  // pairs per warp
+    const int tile = blockIdx.x;
+    const int64_t w0 = (int64_t)tile * kPermTile + (int64_t)warp * kRun;
+    for (int e = threadIdx.x; e < kPermWarps * E; e += kPermThreads) wbase[e] = 0;
+    __syncthreads();
+    griddep_wait();  // the tile counts of the first launch
+    // this warp's counts
+    for (int j = lane; j < kRun; j += 32) {
+        const int64_t i = w0 + j;
+        if (i < n) {
+            const int id = __ldg(ids + i);
+            if (id >= 0 && id < E) atomicAdd(&wbase[warp * E + id], 1);
+        }
+    }
+    // Per expert: pairs in earlier tiles (pre) and in all tiles (tot).  The
+    // [tiles][E] counts sit in L2; to have many loads in flight, thread
+    // (g, c) reads 16-byte column c (4 experts) of every ng-th tile from g,
+    // then the ng partial sums meet in shared memory.
+    if (E % 4 == 0) {
+        const int ncol = E / 4;  // <= 256
+        const int ng = kPermThreads / ncol;
+        int4 pre = make_int4(0, 0, 0, 0), tot = make_int4(0, 0, 0, 0);
+        const int c = threadIdx.x % ncol, g = threadIdx.x / ncol;
+        if (g < ng) {
+            const int4* col = reinterpret_cast<const int4*>(tile_counts) + c;
+#pragma unroll 16
+            for (int j = g; j < ntiles; j += ng) {
+                const int4 v = __ldcg(col + (int64_t)j * ncol);
+                tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
+                if (j < tile) {
+                    pre.x += v.x; pre.y += v.y; pre.z += v.z; pre.w += v.w;
+                }
+            }
+            reinterpret_cast<int4*>(s_part)[g * ncol + c] = pre;
+            reinterpret_cast<int4*>(s_part + 4 * kPermThreads)[g * ncol + c] = tot;
+        }
+        __syncthreads();
+        constexpr int EPT = kPermMaxE / kPermThreads;  // experts per thread, at most
+        int32_t sp[EPT], st[EPT];
+#pragma unroll
+        for (int u = 0; u < EPT; ++u) {
+            const int e = threadIdx.x + u * kPermThreads;
+            sp[u] = 0;
+            st[u] = 0;
+            if (e < E) {
+                for (int q = 0; q < ng; ++q) {
+                    sp[u] += s_part[q * E + e];
+                    st[u] += s_part[4 * kPermThreads + q * E + e];
+                }
+            }
+        }
+        __syncthreads();  // s_pre and s_tot overlay the partial sums
+#pragma unroll
+        for (int u = 0; u < EPT; ++u) {
+            const int e = threadIdx.x + u * kPermThreads;
+            if (e < E) {
+                s_pre[e] = sp[u];
+                s_tot[e] = st[u];
+            }
+        }
+    } else {
+        for (int e = threadIdx.x; e < E; e += kPermThreads) {
+            int32_t pre = 0, post = 0;
+            int j = 0;
+#pragma unroll 8
+            for (; j < tile; ++j) pre += __ldcg(tile_counts + (int64_t)j * E + e);
+#pragma unroll 8
+            for (; j < ntiles; ++j) post += __ldcg(tile_counts + (int64_t)j * E + e);
+            s_pre[e] = pre;
+            s_tot[e] = pre + post;
+        }
+    }
+    __syncthreads();
+    // exclusive scan of the totals over the experts: each thread a contiguous
+    // run of experts, then the runs' sums across the block
+    const int per = (E + kPermThreads - 1) / kPermThreads;
+    const int e0 = threadIdx.x * per, e1 = min(E, e0 + per);
+    int32_t run = 0;
+    for (int e = e0; e < e1; ++e) run += s_tot[e];
+    int32_t incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int32_t wprev = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kPermWarps; ++w) {
+        const int32_t v = s_wsum[w];
+        wprev += w < warp ? v : 0;
+        total += v;
+    }
+    int32_t off = wprev + incl - run;
+    for (int e = e0; e < e1; ++e) {
+        const int32_t c = s_tot[e];
+        if (tile == 0) {
+            counts[e] = c;
+            offsets[e] = off;
+        }
+        s_tot[e] = off;
+        off += c;
+    }
+    if (tile == 0 && threadIdx.x == 0) offsets[E] = total;
+    __syncthreads();
+    // first position of each (warp, expert) of this tile
+    for (int e = threadIdx.x; e < E; e += kPermThreads) {
+        int32_t r = s_tot[e] + s_pre[e];
+        for (int w = 0; w < kPermWarps; ++w) {
+            const int32_t c = wbase[w * E + e];
+            wbase[w * E + e] = r;
+            r += c;
+        }
+    }
+    __syncthreads();
+    // place the warp's pairs in order, 32 at a time
+    const unsigned lt = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < kRun; j0 += 32) {
+        const int64_t i = w0 + j0 + lane;
+        int id = -1;
+        if (i < n) {
+            id = __ldg(ids + i);
+            if (id < 0 || id >= E) {
+                scatter[i] = -1;
+                id = -1;
+            }
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, id);
+        int32_t pos = 0;
+        if (id >= 0) pos = wbase[warp * E + id] + __popc(same & lt);
+        __syncwarp();
+        if (id >= 0) {
+            gather[pos] = (int32_t)i;
+            scatter[i] = pos;
+            if (gate) gate[pos] = __ldg(weights + i);
+            if ((same >> lane) == 1u) wbase[warp * E + id] = pos + 1;  // the group's last lane
+        }
+        __syncwarp();
+    }
 }
 
 // One block of E32 x Q threads (E32 = E rounded up to a warp, Q = 1024 / E32
@@ -242,11 +416,32 @@ int moe_expert_permutation(const int32_t* topk_ids, const float* topk_weights, i
     }
     int32_t* tiles = static_cast<int32_t*>(workspace);
     const int ntiles = (int)perm_tiles(n);
-    perm_hist_kernel<<<ntiles, kPermThreads, 0, st>>>(topk_ids, n, E, tiles);
-    const int e32 = ((E + 31) / 32) * 32;
-    perm_scan_kernel<<<1, e32 * (kPermMaxE / e32), 0, st>>>(tiles, ntiles, E, expert_counts, expert_offsets);
-    perm_scatter_kernel<<<ntiles, kPermThreads, sizeof(int32_t) * kPermWarps * E, st>>>(
-        topk_ids, topk_weights, n, E, tiles, gather_indx, scatter_indx, gate_scal);
+    perm_count_kernel<<<ntiles, kPermThreads, 0, st>>>(topk_ids, n, E, tiles);
+    if (ntiles > kPermPlaceMaxTiles || (reinterpret_cast<uintptr_t>(workspace) % 16) != 0) {
+        // many tiles: one scan block instead of every block summing all tiles
+        // (also for a workspace that 16-byte loads cannot read)
+        const int e32 = ((E + 31) / 32) * 32;
+        perm_scan_kernel<<<1, e32 * (kPermMaxE / e32), 0, st>>>(tiles, ntiles, E, expert_counts, expert_offsets);
+        perm_scatter_kernel<<<ntiles, kPermThreads, sizeof(int32_t) * kPermWarps * E, st>>>(
+            topk_ids, topk_weights, n, E, tiles, gather_indx, scatter_indx, gate_scal);
+    } else {
+        const size_t smem = sizeof(int32_t) * (size_t)kPermWarps * E;
+        // at most 8 * 1024 int32 = 32 KB, plus 8 KB static: within the default limit
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)ntiles, 1, 1);
+        cfg.blockDim = dim3((unsigned)kPermThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t err = cudaLaunchKernelEx(&cfg, perm_place_kernel, topk_ids, topk_weights, n, E, ntiles,
+                                 static_cast<const int32_t*>(tiles), expert_counts, expert_offsets, gather_indx,
+                                 scatter_indx, gate_scal);
+        if (err != cudaSuccess) return set_cuda_error(err, "moe_expert_permutation: launch");
+    }
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return set_cuda_error(err, "moe_expert_permutation: launch");
     return MOE_OK;

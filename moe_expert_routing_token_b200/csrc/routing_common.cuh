@@ -33,6 +33,11 @@ struct RouteArgs {
     int32_t* ids;         // (M, K) int32
     int bias_bf16 = 0;    // 1: round the bias to bf16 before use (the aiter variant)
     float softcap = 0.0f; // softmax: weights from c * tanh(x / c) (0: none)
+    // Partial-logit input (fused router, decode batches): `logits` holds
+    // nparts fp32 partial sums, part_stride floats apart, added in order.
+    int nparts = 0;
+    int64_t part_stride = 0;
+    float* logits_out = nullptr;  // (M, E) fp32 copy of the summed logits, or nullptr
 };
 
 

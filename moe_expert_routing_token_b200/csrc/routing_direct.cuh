@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kDirectThreads)
     constexpr int C = S::C, R = S::R, L = S::L, D = kDirectStages, EPC = S::EPC, CH = S::CH;
     constexpr bool GROUPED = GS > 0;
     constexpr int NG = GROUPED ? C / GS : 1;  // groups per lane
-    static_assert(!GROUPED || (C % GS == 0 && NG <= 4), "a lane owns whole groups");
+    static_assert(!GROUPED || (C % (GS > 0 ? GS : 1) == 0 && NG <= 4), "a lane owns whole groups");
     static_assert(MODE != kKeyApprox || (SCORE == kSigmoid && !GROUPED), "approximate keys: sigmoid, all groups");
 
     extern __shared__ uint8_t smem_raw[];
@@ -306,7 +306,6 @@ __global__ void __launch_bounds__(kDirectThreads)
     const int64_t gw = (int64_t)blockIdx.x * kDirectWarps + warp;
 
 
-    ptx::griddep_launch_dependents();
     if (lane == 0) {
 #pragma unroll
         for (int d = 0; d < D; ++d) ptx::mbar_init(&my_bars[d], 1);
@@ -784,6 +783,9 @@ __global__ void __launch_bounds__(kDirectThreads)
         const int64_t next = gw + (int64_t)(j + D) * nwarps;
         if (lane == 0 && next < n_oct) issue(next, d);
     }
+    // The next kernel in the stream launches once every warp is done: its
+    // blocks would otherwise wait on these SMs and take issue slots.
+    ptx::griddep_launch_dependents();
 }
 
 }  // namespace moe

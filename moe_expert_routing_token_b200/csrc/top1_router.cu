@@ -15,11 +15,13 @@
 // them, and the weight, which depends only on the capped values, is the same
 // whichever of them is chosen.
 //
+// This kernel serves the (K, E) weight layout and hidden sizes that are not
+// a multiple of 64; the rest goes to the tensor-core kernel (top1_tc.cu).
 // With E <= 8 experts the work is 2 * E flops per 2-byte hidden value, below
-// the B200's fp32 CUDA-core ridge (about 11 flops per byte), so one kernel
-// serves every batch size.  At E = 8 the instruction issue (the FMAs plus the
-// bf16 unpacking) is close to the rate at which HBM delivers the hidden
-// states, so E = 8 sits near the balance of the two.  Each 128-thread block takes
+// the B200's fp32 CUDA-core ridge (about 11 flops per byte), but the
+// instruction issue (the FMAs plus the bf16 unpacking) is close to the rate
+// at which HBM delivers the hidden states at E = 8 (measured: 1.1 TB/s at
+// M = 8192, against 4.9 TB/s for the tensor-core kernel).  Each 128-thread block takes
 // 4 rows at a time; every thread walks 8-value chunks of the hidden size,
 // loads the chunk's weights once (E 16-byte vectors, cached in L1/L2) and
 // applies them to the 4 rows.  The partial sums meet through warp shuffles
@@ -38,6 +40,8 @@ namespace moe {
 int set_error(int status, const char* msg);
 int set_cuda_error(cudaError_t err, const char* what);
 int sm_count(int* dev, int* sms);
+int launch_top1_tc(const void* h, const void* w, int64_t M, int K, int E, float softcap, float* weights,
+                   int32_t* ids, float* logits_out, cudaStream_t st);
 
 namespace {
 
@@ -47,6 +51,8 @@ constexpr int kT1Rows = 4;        // rows sharing each weight chunk
 constexpr int kT1Chunk = 8;       // hidden values per 16-byte load
 constexpr int kT1BlocksPerSm = 4;
 constexpr int kT1MaxE = 8;
+constexpr int kT1TcBlockK = 64;     // its k-block
+constexpr int kT1TcMaxE = 256;      // UMMA N limit for M = 128
 
 // The 8 bf16 values of a 16-byte vector, as fp32.
 __device__ __forceinline__ void unpack8(const uint4 q, float (&x)[kT1Chunk]) {
@@ -211,12 +217,21 @@ int moe_fused_router_top1(const void* hidden_states, const void* router_weight, 
     }
     if (!(softcap == softcap) || softcap > 3.4e38f || softcap < -3.4e38f)
         return set_error(MOE_ERR_INVALID_ARG, "moe_fused_router_top1: softcap is not finite");
-    if (E > kT1MaxE) {
-        std::snprintf(msg, sizeof msg, "moe_fused_router_top1: E=%d; the CUDA-core top-1 router is built for E <= %d",
-                      E, kT1MaxE);
+    // The tensor-core kernel whenever K is a multiple of its 64-wide k-block,
+    // the weights are (E, K) (K-major tiles) and E <= 256.  The page sends
+    // batches below 512 tokens with E <= 8 to the CUDA cores; measured here
+    // at M = 64, K = 7168 the CUDA-core kernel takes 13.7 us (E = 8) and the
+    // tensor-core kernel 5.6 us (E = 16), so the CUDA-core kernel serves only
+    // the (K, E) layout and K not a multiple of 64.
+    const bool tc = K % kT1TcBlockK == 0 && weight_layout == MOE_WEIGHT_E_BY_K && E <= kT1TcMaxE;
+    if (!tc && E > kT1MaxE) {
+        std::snprintf(msg, sizeof msg,
+                      "moe_fused_router_top1: E=%d needs the tensor-core kernel: (E, K) weights, K a multiple of "
+                      "%d and E <= %d (got K=%d, layout %d); the CUDA-core kernel takes E <= %d",
+                      E, kT1TcBlockK, kT1TcMaxE, K, weight_layout, kT1MaxE);
         return set_error(MOE_ERR_UNSUPPORTED, msg);
     }
-    if (K % kT1Chunk != 0) {
+    if (!tc && K % kT1Chunk != 0) {
         std::snprintf(msg, sizeof msg, "moe_fused_router_top1: K=%d is not a multiple of %d", K, kT1Chunk);
         return set_error(MOE_ERR_UNSUPPORTED, msg);
     }
@@ -231,6 +246,7 @@ int moe_fused_router_top1(const void* hidden_states, const void* router_weight, 
                          "outputs 4-byte aligned");
     const bool w_ke = weight_layout == MOE_WEIGHT_K_BY_E;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (tc) return launch_top1_tc(hidden_states, router_weight, M, K, E, softcap, topk_weights, topk_ids, logits_out, st);
     switch (E) {
         case 1: return launch_top1<1>(w_ke, hidden_states, router_weight, M, K, softcap, topk_weights, topk_ids, logits_out, st);
         case 2: return launch_top1<2>(w_ke, hidden_states, router_weight, M, K, softcap, topk_weights, topk_ids, logits_out, st);

@@ -266,10 +266,12 @@ def fused_router_topk(hidden_states: torch.Tensor, router_weight: torch.Tensor, 
 
 def fused_router_top1(hidden_states: torch.Tensor, router_weight: torch.Tensor, softcap: float = 0.0,
                       weight_layout: str = "ek", return_logits: bool = False, out=None):
-    """Router projection, softcapping and top-1 on the CUDA cores, for E <= 8
-    experts (moe_fused_router_top1).  ``weight_layout`` "ek": router_weight
-    is (E, K); "ke": (K, E).  Returns (weights (M, 1) fp32, ids (M, 1) int32)
-    or, with ``return_logits``, also the raw fp32 logits (M, E)."""
+    """Router projection, softcapping and top-1 (moe_fused_router_top1): the
+    tensor-core kernel for the "ek" layout with K % 64 == 0 and E <= 256,
+    else the CUDA-core kernel (E <= 8).  ``weight_layout`` "ek":
+    router_weight is (E, K); "ke": (K, E).  Returns (weights (M, 1) fp32,
+    ids (M, 1) int32) or, with ``return_logits``, also the raw fp32 logits
+    (M, E)."""
     _cuda_2d(hidden_states, "hidden_states")
     _cuda_2d(router_weight, "router_weight")
     if hidden_states.dtype != torch.bfloat16 or router_weight.dtype != torch.bfloat16:

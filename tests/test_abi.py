@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.moe_abi_version() == 4
+    assert lib.moe_abi_version() == 5
     assert lib.moe_status_string(0) == b"MOE_OK"
     assert lib.moe_status_string(1) == b"MOE_ERR_INVALID_ARG"
     assert lib.moe_status_string(2) == b"MOE_ERR_UNSUPPORTED"
@@ -110,8 +110,11 @@ def test_top1_router_validation(lib):
     assert lib.moe_fused_router_top1(P, P, 2, 4, 64, 8, 0.0, P, P, None, None) == 1       # layout
     assert lib.moe_fused_router_top1(P, P, 1, 4, 64, 8, float("nan"), P, P, None, None) == 1
     assert b"softcap" in lib.moe_last_error()
-    assert lib.moe_fused_router_top1(P, P, 1, 4, 64, 9, 0.0, P, P, None, None) == 2       # E > 8
-    assert b"E <= 8" in lib.moe_last_error()
+    # E > 8 only on the tensor-core kernel: (E, K) layout, K % 64 == 0, E <= 256
+    assert lib.moe_fused_router_top1(P, P, 0, 4, 64, 9, 0.0, P, P, None, None) == 2       # (K, E) layout
+    assert b"tensor-core" in lib.moe_last_error()
+    assert lib.moe_fused_router_top1(P, P, 1, 4, 72, 9, 0.0, P, P, None, None) == 2       # K % 64
+    assert lib.moe_fused_router_top1(P, P, 1, 4, 64, 257, 0.0, P, P, None, None) == 2     # E > 256
     assert lib.moe_fused_router_top1(P, P, 1, 4, 60, 8, 0.0, P, P, None, None) == 2       # K % 8
     assert lib.moe_fused_router_top1(None, P, 1, 4, 64, 8, 0.0, P, P, None, None) == 1    # null
     assert lib.moe_fused_router_top1(P + 8, P, 1, 4, 64, 8, 0.0, P, P, None, None) == 1   # 16-B alignment

@@ -43,6 +43,13 @@ def test_random_ids(M, k, E, with_weights):
     _check(ids, E, w)
 
 
+@pytest.mark.parametrize("M,k,E", [(65536, 8, 256),    # 512 tiles of 1024 pairs: the two-launch path
+                                   (65537, 8, 256),    # 513 tiles: count, scan, scatter
+                                   (40000, 16, 64)])   # 625 tiles, few experts
+def test_tile_count_paths(M, k, E):
+    _check(_random_ids(M, k, E, seed=M + k), E, torch.rand(M, k, generator=torch.Generator().manual_seed(k)))
+
+
 def test_repeated_ids_and_one_hot_expert():
     _check(_random_ids(777, 5, 12, seed=3, distinct=False), 12)
     _check(torch.full((513, 4), 3, dtype=torch.int32), 8, torch.rand(513, 4))
@@ -78,5 +85,17 @@ def test_deterministic_with_reused_workspace():
     ws = torch.full((need,), 0xAB, dtype=torch.uint8, device=DEV)   # no initial contents needed
     a = _check(ids, 256, workspace=ws)
     b = _check(ids, 256, workspace=ws)
+    for x, y in zip(a[:4], b[:4]):
+        assert torch.equal(x, y)
+
+
+def test_workspace_not_16_byte_aligned():
+    """A workspace that 16-byte loads cannot read takes the three-launch path;
+    the result is the same."""
+    ids = _random_ids(3000, 8, 256, seed=12)
+    need = moe.expert_permutation_workspace_size(3000, 8, 256)
+    buf = torch.full((need + 16,), 0xCD, dtype=torch.uint8, device=DEV)
+    a = _check(ids, 256, workspace=buf[4:4 + need])
+    b = _check(ids, 256)
     for x, y in zip(a[:4], b[:4]):
         assert torch.equal(x, y)

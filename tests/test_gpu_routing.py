@@ -84,7 +84,8 @@ def test_other_dtype(name, M):
     check(op, x, d["bias"], k, renorm, G, TG, rsf)
 
 
-# (op, E, G, TG, k, renorm, rsf, bias) across the three kernel families
+# (op, E, G, TG, k, renorm, rsf, bias) across the kernel families (M = 531 takes the
+# warp-per-row kernel for E = 160 and 256 with G dividing 32)
 SHAPES = [
     ("sigmoid", 256, 8, 4, 8, True, 2.5, True),    # segment, DeepSeek-V3
     ("sigmoid", 256, 4, 2, 6, False, 1.0, True),   # segment, 2 lanes per group
@@ -105,6 +106,9 @@ SHAPES = [
     ("softmax", 1024, 32, 8, 16, False, 1.0, False),  # generic, large
     ("sigmoid", 256, 16, 4, 8, True, 2.5, True),   # generic (lanes would straddle groups)
     ("sigmoid", 72, 9, 3, 6, True, 1.0, True),     # generic, odd group count
+    ("sigmoid", 256, 32, 8, 8, True, 2.5, True),   # one lane per group (warp-per-row kernel)
+    ("softmax", 160, 16, 4, 6, True, 1.0, False),  # two lanes per group of 10
+    ("sigmoid", 160, 32, 6, 8, False, 1.0, True),  # groups of 5 experts, one lane each
 ]
 
 
