@@ -3,13 +3,15 @@
 // followed by its §4 biased grouped top-k, in two launches shaped for latency.
 //
 //  1. fused_decode_proj_kernel: the hidden size is cut into nsplit ranges of
-//     k-blocks, one CTA each (no clusters).  Warp 0 streams the hidden tile
-//     (128 x 64, K-major) and the weight tile (256 x 64, K-major for (E, K)
-//     weights, MN-major for (K, E)) with TMA into a 4-stage ring; warp 1
-//     issues tcgen05.mma (M = 128, N = 256, K = 16) into 256 TMEM columns;
-//     warps 2-5 read the accumulator rows of the batch (one TMEM lane per
-//     thread) and store them, fp32, to the workspace as partial logits
-//     [nsplit][M][256].
+//     k-blocks and the 256 experts into 4 slices of 64, one CTA per (range,
+//     slice) (no clusters): each CTA does a quarter of the tensor work of a
+//     full-width split, so 4x as many SMs share the projection.  Warp 0
+//     streams the hidden tile (128 x 64, K-major) and the weight slice
+//     (64 x 64, K-major for (E, K) weights, MN-major for (K, E)) with TMA into
+//     a 4-stage ring; warp 1 issues tcgen05.mma (M = 128, N = 64, K = 16) into
+//     64 TMEM columns; warps 2-5 read the accumulator rows of the batch (one
+//     TMEM lane per thread) and store them, fp32, to the workspace as partial
+//     logits [nsplit][M][256] (this slice's 64 columns).
 //  2. route_warp_kernel with partial inputs (programmatic dependent launch):
 //     one block per token row; its 4 warps each add a quarter of the nsplit
 //     partials, the quarters are added in warp order (a fixed order, so the
@@ -38,7 +40,9 @@ static __device__ unsigned int g_watchdog_trips_decode;
 namespace {
 
 constexpr int kDBM = 128;
-constexpr int kDBN = 256;
+constexpr int kDE = 256;     // experts (columns of a partial row)
+constexpr int kDBN = 64;     // experts per CTA (N of the MMA)
+constexpr int kDSlices = kDE / kDBN;
 constexpr int kDBK = 64;
 constexpr int kDStages = 4;
 constexpr int kDABytes = kDBM * kDBK * 2;
@@ -72,7 +76,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int split = blockIdx.x;
+    const int split = blockIdx.x / kDSlices;
+    const int n0 = (blockIdx.x % kDSlices) * kDBN;  // first expert of this CTA's slice
     const int kb0 = split * da.kbps;
     int nkb = da.num_kb - kb0;
     if (nkb > da.kbps) nkb = da.kbps;
@@ -119,13 +124,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 const int kc = (kb0 + kb) * kDBK;
                 ptx::mbar_arrive_expect_tx(&full[s], kDStageBytes);
                 ptx::tma_load_2d(a_s, &tmA, kc, 0, &full[s], pol_a);
-                if constexpr (B_MN) {
-#pragma unroll
-                    for (int j = 0; j < kDBN / 64; ++j)
-                        ptx::tma_load_2d(b_s + j * 8192, &tmB, j * 64, kc, &full[s], pol_b);
-                } else {
-                    ptx::tma_load_2d(b_s, &tmB, kc, 0, &full[s], pol_b);
-                }
+                if constexpr (B_MN)
+                    ptx::tma_load_2d(b_s, &tmB, n0, kc, &full[s], pol_b);  // 64 experts x 64 k, MN-major
+                else
+                    ptx::tma_load_2d(b_s, &tmB, kc, n0, &full[s], pol_b);  // 64 experts x 64 k, K-major
             }
             // leave only once the copies issued have landed (bounded)
             for (int k = 0; k < kDStages && k < kb; ++k) {
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
         // no valid logits for the batch, and the watchdog counts the event.
         const bool bad = *s_abort != 0;
         if (__any_sync(kFullMask, r < da.M)) {
-            float* dst = da.ws + ((size_t)split * da.M + r) * kDBN;
+            float* dst = da.ws + ((size_t)split * da.M + r) * kDE + n0;
 #pragma unroll 1
             for (int c0 = 0; c0 < kDBN; c0 += 64) {
                 float v[64];
@@ -206,7 +208,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
 // within kDecodeMaxWs, and no CTA without k-blocks.
 void decode_split(int64_t M, int num_kb, int* nsplit, int* kbps) {
     int target = (num_kb + kDecodeKbPerCta - 1) / kDecodeKbPerCta;
-    const int64_t cap = (int64_t)(kDecodeMaxWs / ((size_t)M * kDBN * sizeof(float)));
+    const int64_t cap = (int64_t)(kDecodeMaxWs / ((size_t)M * kDE * sizeof(float)));
     if (target > cap) target = (int)cap;
     if (target > kDecodeMaxSplit) target = kDecodeMaxSplit;
     if (target < 1) target = 1;
@@ -254,13 +256,21 @@ int launch_decode_route(const RouteArgs& ra, cudaStream_t st) {
 size_t fused_decode_workspace_bytes(int64_t M, int num_kb) {
     int nsplit = 1, kbps = 1;
     decode_split(M, num_kb, &nsplit, &kbps);
-    return (size_t)nsplit * (size_t)M * kDBN * sizeof(float);
+    return (size_t)nsplit * (size_t)M * kDE * sizeof(float);
 }
 
-int launch_fused_decode(const CUtensorMap& tmA, const CUtensorMap& tmB, bool b_mn, const RouteArgs& route,
+int launch_fused_decode(const CUtensorMap& tmA, const void* router_weight, bool b_mn, const RouteArgs& route,
                         float* logits_out, int num_kb, void* workspace, cudaStream_t st) {
     int nsplit = 1, kbps = 1;
     decode_split(route.M, num_kb, &nsplit, &kbps);
+    // the weight in 64 x 64 boxes: (K, E) rows of 64 experts, or (E, K) rows of 64 k
+    const uint64_t K = (uint64_t)num_kb * kDBK;
+    CUtensorMap tmB;
+    cudaError_t terr = b_mn ? encode_tmap_2d(&tmB, router_weight, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, kDE,
+                                             (uint64_t)kDE * 2, 64, kDBK, true)
+                            : encode_tmap_2d(&tmB, router_weight, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDE, K, K * 2,
+                                             kDBK, kDBN, true);
+    if (terr != cudaSuccess) return set_cuda_error(terr, "cuTensorMapEncodeTiled(router_weight, decode)");
     DecodeArgs da;
     da.M = route.M;
     da.num_kb = num_kb;
@@ -272,7 +282,7 @@ int launch_fused_decode(const CUtensorMap& tmA, const CUtensorMap& tmB, bool b_m
         int rc = set_kernel_smem(fn, kDSmem, "cudaFuncSetAttribute(fused router decode smem)");
         if (rc != MOE_OK) return rc;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)nsplit, 1, 1);
+        cfg.gridDim = dim3((unsigned)(nsplit * kDSlices), 1, 1);
         cfg.blockDim = dim3(kDThreads, 1, 1);
         cfg.dynamicSmemBytes = kDSmem;
         cfg.stream = st;
@@ -288,7 +298,7 @@ int launch_fused_decode(const CUtensorMap& tmA, const CUtensorMap& tmB, bool b_m
     RouteArgs ra = route;
     ra.logits = workspace;
     ra.nparts = nsplit;
-    ra.part_stride = route.M * kDBN;
+    ra.part_stride = route.M * kDE;
     ra.logits_out = logits_out;
     const bool grouped = ra.G > 1 && ra.TG < ra.G;
     if (ra.bias)

@@ -16,7 +16,8 @@
 //               distributed shared memory (each CTA of the cluster owns
 //               128/SPLIT rows and receives the other CTAs' partials for
 //               them), summed in a fixed rank order, staged in shared memory
-//               and routed one row per warp by the warp-per-row routing body.
+//               and routed by the same SegRouter body as the segment routing
+//               kernel (8 lanes per row, 4 rows per warp in one pass).
 // The K dimension is split across the SPLIT CTAs of a cluster so that enough
 // SMs stream the hidden states (M=8192: 64 tiles x 2 = 128 CTAs).  A single
 // tile with a long K (decode batches, M <= 128) takes fused_decode.cu
@@ -29,7 +30,6 @@
 #include "fused_router.cuh"
 #include "moe_routing.h"
 #include "routing_kernels.cuh"
-#include "routing_warp.cuh"
 #include "sm100_ptx.cuh"
 #include "tma_host.cuh"
 
@@ -81,6 +81,20 @@ constexpr size_t kOverlayBytes = (size_t)kStages * kStageBytes > kPairExchangeBy
 __host__ __device__ constexpr size_t fused_smem_bytes() {
     return 1024 + kOverlayBytes + Router::BIAS_FLOATS * 4 + 256;
 }
+
+// Owner-side staged logits row: chunk c (32 floats) at c * 36.
+__device__ __forceinline__ int fin_off(int r, int col) { return r * kFinStride + (col >> 5) * 36 + (col & 31); }
+
+template <int SPLIT>
+struct FinScores {
+    const float* fin;
+    int warp_row0;
+    __device__ __forceinline__ void store(int, float, float, float, float) const {}
+    __device__ __forceinline__ float get(int seg, int e) const {
+        const int r = warp_row0 + seg;  // rows past the owned range are padding
+        return r < kBM / SPLIT ? sigmoid_f32(fin[fin_off(r, e)]) : 0.0f;
+    }
+};
 
 template <int SPLIT, bool B_MN_MAJOR, bool BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -381,33 +395,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_dealloc(tmem, 256);
     }
 
-    // Routing of the owned rows: one warp per row (the warp-per-row routing
-    // kernel's body), the epilogue warps taking rows ew, ew + 16, ...
+    // Routing of the owned rows by the epilogue warps (4 rows each per pass).
     if (epi) {
         const bool aborted = *s_abort || *s_peer_abort;
         const int ew = warp - 2;
-        auto* wscr = reinterpret_cast<WarpRowScratch*>(scratch) + ew;
-        static_assert(kEpiWarps * sizeof(WarpRowScratch) <= kEpiWarps * sizeof(typename R_t::Scratch),
-                      "warp routing scratch");
-        // lane l holds experts [8 l, 8 l + 8): chunk l / 4 of the staged row
-        const int loff = (lane >> 2) * 36 + (lane & 3) * 8;
-        float bl[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) bl[c] = BIAS ? s_bias[(lane >> 2) * Router::CS + (lane & 3) * 8 + c] : 0.0f;
-        const bool grouped = fa.route.G > 1 && fa.route.TG < fa.route.G;
-        for (int lr = ew; lr < ROWS; lr += kEpiWarps) {
+        const int seg = lane / R_t::L;
+        const int e0 = (lane % R_t::L) * 32;
+        for (int base = 0; base < ROWS; base += kEpiWarps * R_t::R) {
+            const int warp_row0 = base + ew * R_t::R;
+            const int lr = warp_row0 + seg;
             const int64_t grow = row_base + lr;
-            if (grow >= fa.route.M) break;  // rows ascend
-            float x[8];
-            const float4* src = reinterpret_cast<const float4*>(fin + (size_t)lr * kFinStride + loff);
-            const float4 v0 = src[0], v1 = src[1];
-            x[0] = v0.x; x[1] = v0.y; x[2] = v0.z; x[3] = v0.w;
-            x[4] = v1.x; x[5] = v1.y; x[6] = v1.z; x[7] = v1.w;
-            if (grouped)
-                warp_route_row<256, kSigmoid, BIAS, true>(x, bl, grow, fa.route, *wscr);
-            else
-                warp_route_row<256, kSigmoid, BIAS, false>(x, bl, grow, fa.route, *wscr);
-            if (aborted && lane < fa.route.K) fa.route.ids[grow * fa.route.K + lane] = -1;
+            const bool valid = lr < ROWS && grow < fa.route.M;
+            float x[32];
+            if (lr < ROWS) {
+                const float4* p = reinterpret_cast<const float4*>(fin + fin_off(lr, e0));
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 t = p[i];
+                    x[4 * i] = t.x;
+                    x[4 * i + 1] = t.y;
+                    x[4 * i + 2] = t.z;
+                    x[4 * i + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+            }
+            R_t::route(x, valid, grow, s_bias, scratch[ew], fa.route, FinScores<SPLIT>{fin, warp_row0});
+            if (aborted && valid && (lane % R_t::L) == 0) {
+                for (int t = 0; t < fa.route.K; ++t) fa.route.ids[grow * fa.route.K + t] = -1;
+            }
         }
     }
 }
@@ -655,7 +672,7 @@ int moe_fused_router_topk(const void* hidden_states, const void* router_weight, 
     if (ws_need > 0) {
         // one tile with a long K: split K over CTAs whose partial logits meet
         // in the workspace, then route them (two launches)
-        return launch_fused_decode(tmA, tmB, b_mn, fa.route, logits_out, num_kb, workspace, st);
+        return launch_fused_decode(tmA, router_weight, b_mn, fa.route, logits_out, num_kb, workspace, st);
     }
     if (b_mn)
         return correction_bias ? launch_split<true, true>(split, tmA, tmB, fa, m_tiles, st)

@@ -23,7 +23,7 @@ int route_logits(const void* logits, int dtype, const float* bias, int64_t M, in
 // Decode-sized batches of the fused router (fused_decode.cu): workspace bytes
 // for the partial logits, the two launches, and their watchdog count.
 size_t fused_decode_workspace_bytes(int64_t M, int num_kb);
-int launch_fused_decode(const CUtensorMap& tmA, const CUtensorMap& tmB, bool b_mn, const RouteArgs& route,
+int launch_fused_decode(const CUtensorMap& tmA, const void* router_weight, bool b_mn, const RouteArgs& route,
                         float* logits_out, int num_kb, void* workspace, cudaStream_t st);
 int read_decode_watchdog(unsigned int* count);
 

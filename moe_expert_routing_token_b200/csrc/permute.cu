@@ -30,6 +30,8 @@
 #include <stdint.h>
 
 #include <cstdio>
+#include <mutex>
+#include <unordered_map>
 
 #include "moe_routing.h"
 
@@ -48,6 +50,8 @@ constexpr int kPermMaxE = 1024;
 // counts itself (tiles x E reads per block, from L2); beyond it a single scan
 // block does (three launches).
 constexpr int kPermPlaceMaxTiles = 512;
+// Dynamic shared memory of the placing launch when it stages the tile counts.
+constexpr size_t kPermStageBytes = 192 * 1024;
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
@@ -63,20 +67,42 @@ __global__ void __launch_bounds__(kPermThreads) perm_count_kernel(const int32_t*
     // the ids may be written by the previous kernel in the stream
     griddep_wait();
     const int64_t t0 = (int64_t)blockIdx.x * kPermTile;
-    for (int j = threadIdx.x; j < kPermTile; j += kPermThreads) {
-        const int64_t i = t0 + j;
-        if (i < n) {
-            const int id = __ldg(ids + i);
-            if (id >= 0 && id < E) atomicAdd(&h[id], 1);
-        }
+    constexpr int kPer = kPermTile / kPermThreads;  // pairs per thread, loaded before any is counted
+    int idv[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int64_t i = t0 + threadIdx.x + u * kPermThreads;
+        idv[u] = i < n ? __ldg(ids + i) : -1;
     }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u)
+        if (idv[u] >= 0 && idv[u] < E) atomicAdd(&h[idv[u]], 1);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += kPermThreads) tile_counts[(int64_t)blockIdx.x * E + e] = h[e];
 }
 
+// 16-byte asynchronous copy global -> shared (through L2), and the wait for
+// all of this thread's copies.
+__device__ __forceinline__ void cp_async16(int32_t* dst, const int32_t* src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// 16-byte load through L2 (the tile counts were written by the previous
+// kernel); volatile so that a batch of them is issued before any is used.
+__device__ __forceinline__ int4 ldcg_v4(const int4* p) {
+    int4 v;
+    asm volatile("ld.global.cg.v4.s32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 __global__ void __launch_bounds__(kPermThreads)
     perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ weights, int64_t n, int E,
-                      int ntiles, const int32_t* __restrict__ tile_counts, int32_t* __restrict__ counts,
+                      int ntiles, int stage_counts, const int32_t* __restrict__ tile_counts,
+                      int32_t* __restrict__ counts,
                       int32_t* __restrict__ offsets, int32_t* __restrict__ gather, int32_t* __restrict__ scatter,
                       float* __restrict__ gate) {
     extern __shared__ int32_t wbase[];            // [kPermWarps][E]: next position per (warp, expert)
@@ -93,31 +119,65 @@ __global__ void __launch_bounds__(kPermThreads)
     for (int e = threadIdx.x; e < kPermWarps * E; e += kPermThreads) wbase[e] = 0;
     __syncthreads();
     griddep_wait();  // the tile counts of the first launch
-    // this warp's counts
-    for (int j = lane; j < kRun; j += 32) {
-        const int64_t i = w0 + j;
-        if (i < n) {
-            const int id = __ldg(ids + i);
-            if (id >= 0 && id < E) atomicAdd(&wbase[warp * E + id], 1);
-        }
+    // this warp's pairs, ids and weights loaded at once, then its counts
+    constexpr int kPieces = kRun / 32;
+    int idv[kPieces];
+    float wv[kPieces];
+#pragma unroll
+    for (int u = 0; u < kPieces; ++u) {
+        const int64_t i = w0 + u * 32 + lane;
+        idv[u] = i < n ? __ldg(ids + i) : -1;
+        if (idv[u] < 0 || idv[u] >= E) idv[u] = (i < n) ? -2 : -1;  // -2: out of range, -1: past the batch
+        wv[u] = (gate != nullptr && idv[u] >= 0) ? __ldg(weights + i) : 0.0f;
     }
+#pragma unroll
+    for (int u = 0; u < kPieces; ++u)
+        if (idv[u] >= 0) atomicAdd(&wbase[warp * E + idv[u]], 1);
     // Per expert: pairs in earlier tiles (pre) and in all tiles (tot).  The
     // [tiles][E] counts sit in L2; to have many loads in flight, thread
     // (g, c) reads 16-byte column c (4 experts) of every ng-th tile from g,
     // then the ng partial sums meet in shared memory.
-    if (E % 4 == 0) {
+    if (stage_counts) {
+        // All tile counts into shared memory by asynchronous 16-byte copies
+        // (every copy in flight at once, no registers held), then per-expert
+        // sums from there.
+        int32_t* s_counts = wbase + kPermWarps * E;  // [ntiles][E]
+        const int nv = ntiles * E / 4;
+        for (int v = threadIdx.x; v < nv; v += kPermThreads) cp_async16(s_counts + 4 * v, tile_counts + 4 * v);
+        cp_async_wait_all();
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += kPermThreads) {
+            int32_t pre = 0, post = 0;
+            int j = 0;
+            for (; j < tile; ++j) pre += s_counts[j * E + e];
+            for (; j < ntiles; ++j) post += s_counts[j * E + e];
+            s_pre[e] = pre;
+            s_tot[e] = pre + post;
+        }
+    } else if (E % 4 == 0) {
         const int ncol = E / 4;  // <= 256
         const int ng = kPermThreads / ncol;
         int4 pre = make_int4(0, 0, 0, 0), tot = make_int4(0, 0, 0, 0);
         const int c = threadIdx.x % ncol, g = threadIdx.x / ncol;
         if (g < ng) {
             const int4* col = reinterpret_cast<const int4*>(tile_counts) + c;
-#pragma unroll 16
-            for (int j = g; j < ntiles; j += ng) {
-                const int4 v = __ldcg(col + (int64_t)j * ncol);
-                tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
-                if (j < tile) {
-                    pre.x += v.x; pre.y += v.y; pre.z += v.z; pre.w += v.w;
+            // batches of kBatch loads issued before any is used
+            constexpr int kBatch = 16;
+            for (int j0 = g; j0 < ntiles; j0 += kBatch * ng) {
+                int4 v[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int j = j0 + u * ng;
+                    v[u] = make_int4(0, 0, 0, 0);
+                    if (j < ntiles) v[u] = ldcg_v4(col + (int64_t)j * ncol);
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int j = j0 + u * ng;
+                    tot.x += v[u].x; tot.y += v[u].y; tot.z += v[u].z; tot.w += v[u].w;
+                    if (j < tile) {
+                        pre.x += v[u].x; pre.y += v[u].y; pre.z += v[u].z; pre.w += v[u].w;
+                    }
                 }
             }
             reinterpret_cast<int4*>(s_part)[g * ncol + c] = pre;
@@ -205,16 +265,11 @@ __global__ void __launch_bounds__(kPermThreads)
     __syncthreads();
     // place the warp's pairs in order, 32 at a time
     const unsigned lt = (1u << lane) - 1u;
-    for (int j0 = 0; j0 < kRun; j0 += 32) {
-        const int64_t i = w0 + j0 + lane;
-        int id = -1;
-        if (i < n) {
-            id = __ldg(ids + i);
-            if (id < 0 || id >= E) {
-                scatter[i] = -1;
-                id = -1;
-            }
-        }
+#pragma unroll
+    for (int u = 0; u < kPieces; ++u) {
+        const int64_t i = w0 + u * 32 + lane;
+        const int id = idv[u] >= 0 ? idv[u] : -1;
+        if (idv[u] == -2) scatter[i] = -1;
         const unsigned same = __match_any_sync(0xffffffffu, id);
         int32_t pos = 0;
         if (id >= 0) pos = wbase[warp * E + id] + __popc(same & lt);
@@ -222,7 +277,7 @@ __global__ void __launch_bounds__(kPermThreads)
         if (id >= 0) {
             gather[pos] = (int32_t)i;
             scatter[i] = pos;
-            if (gate) gate[pos] = __ldg(weights + i);
+            if (gate) gate[pos] = wv[u];
             if ((same >> lane) == 1u) wbase[warp * E + id] = pos + 1;  // the group's last lane
         }
         __syncwarp();
@@ -425,8 +480,26 @@ int moe_expert_permutation(const int32_t* topk_ids, const float* topk_weights, i
         perm_scatter_kernel<<<ntiles, kPermThreads, sizeof(int32_t) * kPermWarps * E, st>>>(
             topk_ids, topk_weights, n, E, tiles, gather_indx, scatter_indx, gate_scal);
     } else {
-        const size_t smem = sizeof(int32_t) * (size_t)kPermWarps * E;
-        // at most 8 * 1024 int32 = 32 KB, plus 8 KB static: within the default limit
+        // Stage every tile's counts in shared memory when they fit (with the
+        // warps' cursors, at most kPermStageBytes); else sum them from L2.
+        const size_t cursors = sizeof(int32_t) * (size_t)kPermWarps * E;
+        const size_t staged = sizeof(int32_t) * (size_t)ntiles * E;
+        const int stage = (E % 4 == 0 && cursors + staged <= kPermStageBytes) ? 1 : 0;
+        const size_t smem = cursors + (stage ? staged : 0);
+        if (stage) {  // dynamic + static shared memory may exceed the default 48 KB
+            static std::mutex mu;
+            static std::unordered_map<int, bool> done;  // device ordinal -> attribute set
+            int dev = 0;
+            cudaError_t e0 = cudaGetDevice(&dev);
+            if (e0 != cudaSuccess) return set_cuda_error(e0, "moe_expert_permutation: cudaGetDevice");
+            std::lock_guard<std::mutex> lk(mu);
+            if (!done[dev]) {
+                e0 = cudaFuncSetAttribute(perm_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)kPermStageBytes);
+                if (e0 != cudaSuccess) return set_cuda_error(e0, "moe_expert_permutation: kernel attribute");
+                done[dev] = true;
+            }
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)ntiles, 1, 1);
         cfg.blockDim = dim3((unsigned)kPermThreads, 1, 1);
@@ -437,7 +510,7 @@ int moe_expert_permutation(const int32_t* topk_ids, const float* topk_weights, i
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaError_t err = cudaLaunchKernelEx(&cfg, perm_place_kernel, topk_ids, topk_weights, n, E, ntiles,
+        cudaError_t err = cudaLaunchKernelEx(&cfg, perm_place_kernel, topk_ids, topk_weights, n, E, ntiles, stage,
                                  static_cast<const int32_t*>(tiles), expert_counts, expert_offsets, gather_indx,
                                  scatter_indx, gate_scal);
         if (err != cudaSuccess) return set_cuda_error(err, "moe_expert_permutation: launch");

@@ -277,6 +277,10 @@ __global__ void __launch_bounds__(kWarpRowThreads) route_warp_kernel(RouteArgs a
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * kWarpRowWarps;
 
+    // The fused router's decode routing (PARTS) lets its dependent, the next
+    // projection launch, set up at once: those CTAs take a whole SM each and
+    // do not share SMs with this kernel's small blocks.
+    if constexpr (PARTS) ptx::griddep_launch_dependents();
     // Inputs may be written by the previous kernel in the stream: wait for it.
     ptx::griddep_wait();
 
@@ -339,7 +343,7 @@ __global__ void __launch_bounds__(kWarpRowThreads) route_warp_kernel(RouteArgs a
     // Let the next kernel in the stream launch only now: its blocks, waiting
     // on griddepcontrol.wait, would otherwise share this kernel's SMs (small
     // blocks co-reside) and take issue slots from it.
-    ptx::griddep_launch_dependents();
+    if constexpr (!PARTS) ptx::griddep_launch_dependents();
 }
 
 }  // namespace moe
