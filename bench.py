@@ -108,7 +108,7 @@ def workload_desc(name: str, M: int) -> dict:
     elif name == "softmax":
         d["workload"] = f"softmax top-k E=8 k=2 renormalise, M={M}, fp32 logits"
     elif name == "top1":
-        d["workload"] = (f"small-E fused router on the CUDA cores: (M,{sp.K}) bf16 x ({sp.E},{sp.K}) bf16 "
+        d["workload"] = (f"fused top-1 router (tcgen05 projection): (M,{sp.K}) bf16 x ({sp.E},{sp.K}) bf16 "
                          f"weight, softcap {sp.softcap:g}, top-1 with weight 1/sum exp, M={M}")
         d["K"] = sp.K
         d["softcap"] = sp.softcap

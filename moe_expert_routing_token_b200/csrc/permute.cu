@@ -147,12 +147,30 @@ __global__ void __launch_bounds__(kPermThreads)
         cp_async_wait_all();
         __syncthreads();
         for (int e = threadIdx.x; e < E; e += kPermThreads) {
-            int32_t pre = 0, post = 0;
+            // 8 independent partial sums keep 8 shared-memory loads in flight
+            int32_t pre[8] = {0, 0, 0, 0, 0, 0, 0, 0}, tot[8] = {0, 0, 0, 0, 0, 0, 0, 0};
             int j = 0;
-            for (; j < tile; ++j) pre += s_counts[j * E + e];
-            for (; j < ntiles; ++j) post += s_counts[j * E + e];
-            s_pre[e] = pre;
-            s_tot[e] = pre + post;
+            for (; j + 8 <= ntiles; j += 8) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int32_t v = s_counts[(j + u) * E + e];
+                    tot[u] += v;
+                    pre[u] += (j + u < tile) ? v : 0;
+                }
+            }
+            for (; j < ntiles; ++j) {
+                const int32_t v = s_counts[j * E + e];
+                tot[0] += v;
+                pre[0] += (j < tile) ? v : 0;
+            }
+            int32_t sp = 0, st = 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                sp += pre[u];
+                st += tot[u];
+            }
+            s_pre[e] = sp;
+            s_tot[e] = st;
         }
     } else if (E % 4 == 0) {
         const int ncol = E / 4;  // <= 256

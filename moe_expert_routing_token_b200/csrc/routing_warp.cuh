@@ -240,6 +240,8 @@ __device__ __forceinline__ void warp_route_row(const float (&x)[E / 32], const f
             }
         }
     }
+    __syncwarp();  // the output slots are written before they are read
+
     // ---- weights: gather, renormalise, scale, store
     float wv = 0.0f;
     int iv = 0;
