@@ -65,7 +65,7 @@ struct TcRing {
     static constexpr int A_BYTES = kTcBM * kTcBK * 2;
     static constexpr int B_BYTES = NP * kTcBK * 2;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int S = (192 * 1024 / STAGE) < 6 ? (192 * 1024 / STAGE) : 6;  // ring depth
+    static constexpr int S = (192 * 1024 / STAGE) < 10 ? (192 * 1024 / STAGE) : 10;  // ring depth
     static constexpr int TCOLS = NP < 32 ? 32 : NP;  // TMEM columns: a power of two >= 32
     static constexpr int NP32 = (NP + 31) / 32 * 32;
     static_assert(NP % 16 == 0 && NP >= 16 && NP <= 256, "UMMA N for M = 128");
