@@ -21,15 +21,11 @@
 //      a contiguous run of the tile's pairs in order; within a 32-pair piece,
 //      lanes holding the same expert are ranked by __match_any_sync, so pairs
 //      keep their index order.  Block 0 writes counts and offsets.
-// When every tile's block can be resident at once (cooperative launch), the
-// two steps are one launch: each block writes its tile's counts, a grid-wide
-// barrier stands for the launch boundary, and the block goes on to place.
 // With more than kPermPlaceMaxTiles tiles the second step is split in two,
 // so that no block reads every tile's counts: perm_scan_kernel (one block)
 // turns the counts into totals, offsets and each tile's first position per
 // expert, and perm_scatter_kernel places the pairs from those.
 // Ids outside [0, E) are skipped: not counted, scatter_indx = -1.
-#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -103,13 +99,9 @@ __device__ __forceinline__ int4 ldcg_v4(const int4* p) {
     return v;
 }
 
-// COOP: one cooperative launch does the counting too: every block writes
-// its tile's counts, then a grid-wide barrier (all blocks resident) stands
-// where the launch boundary between perm_count_kernel and this kernel is.
-template <bool COOP>
 __global__ void __launch_bounds__(kPermThreads)
     perm_place_kernel(const int32_t* __restrict__ ids, const float* __restrict__ weights, int64_t n, int E,
-                      int ntiles, int stage_counts, int32_t* __restrict__ tile_counts,
+                      int ntiles, int stage_counts, const int32_t* __restrict__ tile_counts,
                       int32_t* __restrict__ counts,
                       int32_t* __restrict__ offsets, int32_t* __restrict__ gather, int32_t* __restrict__ scatter,
                       float* __restrict__ gate) {
@@ -141,16 +133,6 @@ __global__ void __launch_bounds__(kPermThreads)
 #pragma unroll
     for (int u = 0; u < kPieces; ++u)
         if (idv[u] >= 0) atomicAdd(&wbase[warp * E + idv[u]], 1);
-    if constexpr (COOP) {
-        __syncthreads();
-        for (int e = threadIdx.x; e < E; e += kPermThreads) {
-            int32_t c = 0;
-#pragma unroll
-            for (int w = 0; w < kPermWarps; ++w) c += wbase[w * E + e];
-            tile_counts[(int64_t)tile * E + e] = c;
-        }
-        cooperative_groups::this_grid().sync();  // every tile's counts are written
-    }
     // Per expert: pairs in earlier tiles (pre) and in all tiles (tot).  The
     // [tiles][E] counts sit in L2; to have many loads in flight, thread
     // (g, c) reads 16-byte column c (4 experts) of every ng-th tile from g,
@@ -507,10 +489,10 @@ int moe_expert_permutation(const int32_t* topk_ids, const float* topk_weights, i
     }
     int32_t* tiles = static_cast<int32_t*>(workspace);
     const int ntiles = (int)perm_tiles(n);
+    perm_count_kernel<<<ntiles, kPermThreads, 0, st>>>(topk_ids, n, E, tiles);
     if (ntiles > kPermPlaceMaxTiles || (reinterpret_cast<uintptr_t>(workspace) % 16) != 0) {
         // many tiles: one scan block instead of every block summing all tiles
         // (also for a workspace that 16-byte loads cannot read)
-        perm_count_kernel<<<ntiles, kPermThreads, 0, st>>>(topk_ids, n, E, tiles);
         const int e32 = ((E + 31) / 32) * 32;
         perm_scan_kernel<<<1, e32 * (kPermMaxE / e32), 0, st>>>(tiles, ntiles, E, expert_counts, expert_offsets);
         perm_scatter_kernel<<<ntiles, kPermThreads, sizeof(int32_t) * kPermWarps * E, st>>>(
@@ -522,35 +504,18 @@ int moe_expert_permutation(const int32_t* topk_ids, const float* topk_weights, i
         const size_t staged = sizeof(int32_t) * (size_t)ntiles * E;
         const int stage = (E % 4 == 0 && cursors + staged <= kPermStageBytes) ? 1 : 0;
         const size_t smem = cursors + (stage ? staged : 0);
-        int dev = 0, sms = 0;
-        cudaError_t e0 = cudaGetDevice(&dev);
-        if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e0 != cudaSuccess) return set_cuda_error(e0, "moe_expert_permutation: device query");
-        // one cooperative launch when every tile's block can be resident at once
-        bool coop = false;
-        {
+        if (stage) {  // dynamic + static shared memory may exceed the default 48 KB
             static std::mutex mu;
-            static std::unordered_map<int, int> coop_ok;  // device ordinal -> cooperative launch supported
+            static std::unordered_map<int, bool> done;  // device ordinal -> attribute set
+            int dev = 0;
+            cudaError_t e0 = cudaGetDevice(&dev);
+            if (e0 != cudaSuccess) return set_cuda_error(e0, "moe_expert_permutation: cudaGetDevice");
             std::lock_guard<std::mutex> lk(mu);
-            auto it = coop_ok.find(dev);
-            if (it == coop_ok.end()) {
-                int v = 0;
-                e0 = cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, dev);
-                if (e0 != cudaSuccess) return set_cuda_error(e0, "moe_expert_permutation: device query");
-                e0 = cudaFuncSetAttribute(perm_place_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (!done[dev]) {
+                e0 = cudaFuncSetAttribute(perm_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)kPermStageBytes);
-                if (e0 == cudaSuccess)
-                    e0 = cudaFuncSetAttribute(perm_place_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              (int)kPermStageBytes);
                 if (e0 != cudaSuccess) return set_cuda_error(e0, "moe_expert_permutation: kernel attribute");
-                it = coop_ok.emplace(dev, v).first;
-            }
-            if (it->second) {
-                int per_sm = 0;
-                e0 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, perm_place_kernel<true>, kPermThreads,
-                                                                   smem);
-                if (e0 != cudaSuccess) return set_cuda_error(e0, "moe_expert_permutation: occupancy query");
-                coop = (int64_t)per_sm * sms >= ntiles;
+                done[dev] = true;
             }
         }
         cudaLaunchConfig_t cfg = {};
@@ -559,22 +524,13 @@ int moe_expert_permutation(const int32_t* topk_ids, const float* topk_weights, i
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
-        if (coop) {
-            attr[0].id = cudaLaunchAttributeCooperative;
-            attr[0].val.cooperative = 1;
-        } else {
-            perm_count_kernel<<<ntiles, kPermThreads, 0, st>>>(topk_ids, n, E, tiles);
-            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[0].val.programmaticStreamSerializationAllowed = 1;
-        }
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaError_t err = coop ? cudaLaunchKernelEx(&cfg, perm_place_kernel<true>, topk_ids, topk_weights, n, E,
-                                                    ntiles, stage, tiles, expert_counts, expert_offsets,
-                                                    gather_indx, scatter_indx, gate_scal)
-                               : cudaLaunchKernelEx(&cfg, perm_place_kernel<false>, topk_ids, topk_weights, n, E,
-                                                    ntiles, stage, tiles, expert_counts, expert_offsets,
-                                                    gather_indx, scatter_indx, gate_scal);
+        cudaError_t err = cudaLaunchKernelEx(&cfg, perm_place_kernel, topk_ids, topk_weights, n, E, ntiles, stage,
+                                 static_cast<const int32_t*>(tiles), expert_counts, expert_offsets, gather_indx,
+                                 scatter_indx, gate_scal);
         if (err != cudaSuccess) return set_cuda_error(err, "moe_expert_permutation: launch");
     }
     cudaError_t err = cudaGetLastError();
