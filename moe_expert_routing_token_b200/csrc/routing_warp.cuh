@@ -17,11 +17,11 @@
 //    against the G group scores (shuffles from each group's first lane, ties
 //    to the lower group index), and lanes of dropped groups zero their keys
 //    (zero is below every admissible key).
-//  * Threshold.  tau = the k-th largest of the 32 lane maxima, by k rounds
-//    of __reduce_max_sync (each round's lowest maximal lane drops out).  The
-//    maxima are distinct experts, so every expert of the top k has a key >=
-//    tau; those keys (about k + 4 on the benchmark workloads) are the
-//    candidates.
+//  * Threshold.  tau = about the k-th largest of the 32 lane maxima, by k
+//    rounds of __reduce_max_sync on the maxima made unique by the lane index
+//    in their 5 low bits (each round's winner drops out); the maxima are
+//    distinct experts, so every expert of the top k has a key >= tau; those
+//    keys (about k + 4 on the benchmark workloads) are the candidates.
 //  * Rank.  The candidates go to a per-warp list in lane order (positions
 //    from a ballot prefix of the counts); lane t ranks candidate t by
 //    counting the larger keys (16-byte broadcast reads) and writes it to
@@ -147,21 +147,24 @@ __device__ __forceinline__ void warp_route_row(const float (&x)[E / 32], const f
         }
     }
 
-    // ---- threshold: the k-th largest of the 32 lane maxima.  They belong
-    // to distinct experts, so at least k experts have keys >= tau: every
-    // expert of the top k has a key >= tau.
+    // ---- threshold: about the k-th largest of the 32 lane maxima.  Each
+    // lane's maximum, its 5 low bits replaced by 31 - lane, is unique, so one
+    // __reduce_max_sync per round finds the round's largest and its lane,
+    // which drops out.  After k rounds, tau = that value with the 5 low bits
+    // cleared: k distinct experts (the rounds' lane maxima) have keys >= tau,
+    // so every expert of the top k has a key >= tau.
     uint32_t lm = ku[0];
 #pragma unroll
     for (int c = 1; c < C; ++c) lm = max(lm, ku[c]);
     uint32_t tau = 0u;
     {
-        uint32_t v = lm;
+        uint32_t v = (lm & ~31u) | (31u - (uint32_t)lane);
 #pragma unroll 1
         for (int j = 0; j < K; ++j) {
             tau = __reduce_max_sync(kFullMask, v);
-            const unsigned eq = __ballot_sync(kFullMask, v == tau);
-            if (lane == __ffs(eq) - 1) v = 0u;
+            v = (v == tau) ? 0u : v;
         }
+        tau &= ~31u;
     }
     // candidates: admissible keys >= tau
     uint32_t cm = 0u;
