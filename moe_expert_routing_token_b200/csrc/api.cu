@@ -294,10 +294,10 @@ int launch_direct(const RouteArgs& a, cudaStream_t st) {
 }
 
 // Batches up to this size route one row per warp (route_warp_kernel): the
-// shortest chain per row.  Measured on B200 (bf16 E = 256, k = 8): 2.3 us at
-// M = 64 and 5.1 us at M = 4096 (direct kernel: 4.3 and 5.8 us); from
-// M = 8192 the direct kernel's fewer instructions per row win (5.9 against
-// 8.2 us).
+// shortest chain per row.  Measured on B200 (bf16 E = 256, k = 8, sigmoid
+// with bias): 2.1 us at M = 64 and 4.7 us at M = 4096 (direct kernel: 4.3
+// and 5.8 us); from M = 8192 the direct kernel's fewer instructions per row
+// win (5.9 against 8.2 us).
 constexpr int64_t kWarpRowMaxRows = 4096;
 
 template <typename TIn, int E, int SCORE, bool BIAS, bool GROUPED>
@@ -348,8 +348,9 @@ int try_warp_rows(const RouteArgs& a, cudaStream_t st) {
 // the serial work per warp, for latency).
 constexpr int64_t kDirectWideRows = 32768;
 
-// The direct kernel's shapes: E = 256 or 160, topk <= 8, every group kept or
-// 8 groups.  Returns -1 for other shapes.
+// The direct kernel's shapes (instantiated for E = 256; try_direct keeps
+// E = 160 off it): topk <= 8, every group kept or 8 groups.  Returns -1 for
+// other shapes.
 template <typename TIn, int E, int L, int SCORE, bool BIAS>
 int try_direct_el(const RouteArgs& a, cudaStream_t st) {
     constexpr int GS8 = E / 8;  // experts per group with 8 groups

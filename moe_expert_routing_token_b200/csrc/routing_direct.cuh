@@ -5,27 +5,30 @@
 //
 // Every warp is its own producer and consumer; no warp waits for another.
 //
-//  * Staging.  A warp owns "octets" of R = 8 token rows, four lanes per row
-//    and C = E / 4 experts per lane.  One elected lane brings an octet into
+//  * Staging.  A warp owns "octets" of R = 32 / L token rows, L = 4 or 8
+//    lanes per row and C = E / L experts per lane (the library takes L = 8
+//    below 32768 rows, L = 4 above).  One elected lane brings an octet into
 //    shared memory with bulk asynchronous copies completing on the warp's
 //    mbarrier, so the whole octet is in flight with no register cost; a warp
 //    keeps kDirectStages octets in flight, and all loads of a call are issued
 //    at entry when the grid covers the batch.  For E = 256 (rows of 512 or
 //    1024 bytes) one 2-D TMA copy moves the octet, the logits seen as rows of
 //    128 bytes with the 128-byte swizzle: a lane's segment is one or two of
-//    those rows, and the swizzle spreads the four lanes of a row (and the two
-//    rows of a quarter-warp) over distinct bank groups.  For E = 160 each
+//    those rows, and the swizzle spreads the lanes of a row (and the rows
+//    of a quarter-warp) over distinct bank groups.  For E = 160 each
 //    row is copied to a padded shared-memory row (or the octet in one copy
-//    when no padding is needed), which spreads the banks the same way.  The
-//    register order of every lane's experts is its segment order.
+//    when no padding is needed), which spreads the banks the same way (that
+//    shape is built and correct, but the library dispatches E = 160 to the
+//    two-phase streaming kernel, which measured faster).  The register order
+//    of every lane's experts is its segment order.
 //  * Threshold.  Each lane scores its C experts (selection keys), takes the
-//    maxima of blocks of 8 experts, and the row's four lanes find tau, the
+//    maxima of blocks of 8 experts, and the row's L lanes find tau, the
 //    k-th largest of each lane's four largest block maxima, with a merge
 //    network over xor-shuffles: tau is a lower bound for the k-th best key,
 //    since the maxima belong to distinct experts.  With group selection the kept groups are ranked first
 //    and tau is the k-th largest of their top-2 values.
 //  * Candidates.  Experts with key >= tau - band (about 10 per row on the
-//    benchmark workloads) are appended to a per-row list; the row's four
+//    benchmark workloads) are appended to a per-row list; the row's L
 //    lanes then share the list evenly, compute the exact keys of their
 //    entries and rank each one by counting the candidates above it.  The rank
 //    is the output slot, so the ids leave in descending key order.  Exact keys that tie (bf16 logits repeat, so a few rows per
@@ -571,8 +574,8 @@ __global__ void __launch_bounds__(kDirectThreads)
         bool slow = valid && (n > kDirectCap || n < K);
 
         // ---- candidate list: ids first, then exact keys by list position ----
-        // Each lane appends its candidates' ids; then the row's four lanes take
-        // the list entries t = sl, sl + 4, ... (an even share, whatever lane the
+        // Each lane appends its candidates' ids; then the row's L lanes take
+        // the list entries t = sl, sl + L, ... (an even share, whatever lane the
         // experts live in), compute their exact keys and rank them.
         if (!slow) {
             int pos = incl - cnt;
