@@ -343,11 +343,6 @@ int try_warp_rows(const RouteArgs& a, cudaStream_t st) {
     return -1;
 }
 
-// Batches at least this large route bf16 E = 256 rows with 4 lanes per row
-// (fewer instructions per row); smaller ones with 8 (twice the warps, half
-// the serial work per warp, for latency).
-constexpr int64_t kDirectWideRows = 32768;
-
 // The direct kernel's shapes (instantiated for E = 256; try_direct keeps
 // E = 160 off it): topk <= 8, every group kept or 8 groups.  Returns -1 for
 // other shapes.
@@ -365,12 +360,14 @@ int try_direct_el(const RouteArgs& a, cudaStream_t st) {
     return -1;
 }
 
+// Eight lanes per row at every batch size.  Measured on B200 (bf16 E = 256,
+// k = 8, sigmoid with bias): 10.7 / 18.7 us at M = 32768 / 65536 against
+// 11.7 / 19.5 with 4 lanes per row (grouped, G = 8: 13.9 / 25.1 against
+// 15.8 / 27.4).  The four-lane form issues fewer instructions per row but
+// runs half the warps with twice the serial work each.
 template <typename TIn, int E, int SCORE, bool BIAS>
 int try_direct_e(const RouteArgs& a, cudaStream_t st) {
-    if constexpr (sizeof(TIn) == 4) return try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
-    else
-        return a.M >= kDirectWideRows ? try_direct_el<TIn, E, 4, SCORE, BIAS>(a, st)
-                                      : try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
+    return try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
 }
 
 template <typename TIn, int SCORE, bool BIAS>

@@ -6,8 +6,8 @@
 // Every warp is its own producer and consumer; no warp waits for another.
 //
 //  * Staging.  A warp owns "octets" of R = 32 / L token rows, L = 4 or 8
-//    lanes per row and C = E / L experts per lane (the library takes L = 8
-//    below 32768 rows, L = 4 above).  One elected lane brings an octet into
+//    lanes per row and C = E / L experts per lane (the library dispatches
+//    L = 8 at every batch size).  One elected lane brings an octet into
 //    shared memory with bulk asynchronous copies completing on the warp's
 //    mbarrier, so the whole octet is in flight with no register cost; a warp
 //    keeps kDirectStages octets in flight, and all loads of a call are issued
@@ -23,17 +23,21 @@
 //    of every lane's experts is its segment order.
 //  * Threshold.  Each lane scores its C experts (selection keys), takes the
 //    maxima of blocks of 8 experts, and the row's L lanes find tau, the
-//    k-th largest of each lane's four largest block maxima, with a merge
-//    network over xor-shuffles: tau is a lower bound for the k-th best key,
-//    since the maxima belong to distinct experts.  With group selection the kept groups are ranked first
-//    and tau is the k-th largest of their top-2 values.
+//    k-th largest of each lane's two (L = 8) or four (L = 4) largest block
+//    maxima, with a merge network over xor-shuffles: tau is a lower bound
+//    for the k-th best key, since the maxima belong to distinct experts.
+//    With group selection the kept groups are ranked first and tau is the
+//    k-th largest of their block maxima.
 //  * Candidates.  Experts with key >= tau - band (about 10 per row on the
 //    benchmark workloads) are appended to a per-row list; the row's L
 //    lanes then share the list evenly, compute the exact keys of their
 //    entries and rank each one by counting the candidates above it.  The rank
-//    is the output slot, so the ids leave in descending key order.  Exact keys that tie (bf16 logits repeat, so a few rows per
-//    thousand have them) are detected from the rank sum and ranked again with
-//    ties to the lower expert index.  A row with more than kDirectCap
+//    is the output slot, so the ids leave in descending key order.  When no
+//    row of the warp has more than 16 candidates (nearly always), the list
+//    is padded to 16 and ranked in straight-line code: each lane reads the
+//    16 keys once for both of its entries.  Exact keys that tie (bf16
+//    logits repeat, so a few rows per thousand have them) are detected from
+//    the rank sum and ranked again with ties to the lower expert index.  A row with more than kDirectCap
 //    candidates or fewer than k (massive ties, NaN scores) is routed by the
 //    whole warp: E / 32 exact keys per lane and k rounds of warp arg-max.
 //
@@ -61,6 +65,7 @@ static __device__ unsigned int g_watchdog_trips_direct;
 constexpr int kDirectWarps = 4;
 constexpr int kDirectThreads = kDirectWarps * 32;
 constexpr int kDirectCap = 32;     // candidates per row on the fast path
+constexpr int kDirectFastN = 16;   // list length when every row of the warp has at most this many
 constexpr int kDirectStages = 2;   // octets a warp keeps in flight
 
 enum KeyMode : int { kKeyRaw = 0, kKeyApprox = 1, kKeyExact = 2 };
@@ -163,7 +168,8 @@ constexpr size_t direct_smem_bytes() {
     return 1024 + (size_t)kDirectWarps * kDirectStages * S::STAGE +     // staged octets
            (size_t)kDirectWarps * sizeof(DirectLists<S::R>) +          // candidate lists
            (size_t)S::L * S::CS * 4 + (size_t)E * 4 +                  // bias tables
-           (size_t)kDirectWarps * kDirectStages * 8;                   // mbarriers
+           (size_t)kDirectWarps * kDirectStages * 8 +                  // mbarriers
+           (size_t)kDirectWarps * 4;                                   // per-warp max |bias|
 }
 
 // Compare-exchange, descending.
@@ -235,6 +241,36 @@ __device__ __forceinline__ float row_kth(const float (&in)[P], int K, float& vma
     return kth_of_sorted8(a, K);
 }
 
+// As row_kth for eight lanes holding two values each, t0 >= t1: the xor-1
+// exchange makes sorted 4-lists ([t0, t1, p1, p0] is bitonic), the xor-2
+// exchange sorted 8-lists, and the xor-4 exchange the top 8 of the 16 (the
+// elementwise maximum against the reversed partner, a bitonic sequence that
+// is sorted only when K < 8 needs it).
+template <int L>
+__device__ __forceinline__ float row_kth2(float t0, float t1, int K, float& vmax) {
+    static_assert(L == 8, "two values per lane on eight lanes");
+    float a[8];
+    {
+        float x[4] = {t0, t1, __shfl_xor_sync(kFullMask, t1, 1), __shfl_xor_sync(kFullMask, t0, 1)};
+        bitonic_clean_desc(x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            a[i] = x[i];
+            a[7 - i] = __shfl_xor_sync(kFullMask, x[i], 2);
+        }
+        bitonic_clean_desc(a);
+        float b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) b[i] = __shfl_xor_sync(kFullMask, a[i], 4);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], b[7 - i]);
+    }
+    vmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+    if (K == 8) return fminf(fminf(fminf(a[0], a[1]), fminf(a[2], a[3])), fminf(fminf(a[4], a[5]), fminf(a[6], a[7])));
+    bitonic_clean_desc(a);
+    return kth_of_sorted8(a, K);
+}
+
 // Unpack one 16-byte chunk into fp32 values.
 template <typename TIn>
 __device__ __forceinline__ void unpack_chunk(const uint4& v, float* x);
@@ -279,8 +315,19 @@ __device__ __forceinline__ void exact_key(float x, float b, float& key, float& p
 
 // GS: experts per group when groups are selected (the lane owns C / GS whole
 // groups), 0 when every group is kept.
+// Resident blocks per SM the compiler is asked to fit, the most that compile
+// without spills.  Eight lanes per bf16 row: 8 (64 registers) for
+// approximate keys, 7 (72) for the other sigmoid keys, 5 (96) for softmax;
+// at 16384 rows that puts (nearly) one octet per warp in flight.  Other
+// shapes: 4 (128 registers).
+template <typename TIn, int L, int SCORE, int MODE>
+constexpr int direct_min_blocks() {
+    if (sizeof(TIn) != 2 || L != 8) return 4;
+    return SCORE == kSoftmax ? 5 : (MODE == kKeyApprox ? 8 : 7);
+}
+
 template <typename TIn, int E, int L_, int SCORE, bool BIAS, int MODE, int GS>
-__global__ void __launch_bounds__(kDirectThreads)
+__global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCORE, MODE>())
     route_direct_kernel(const __grid_constant__ CUtensorMap tmap, RouteArgs a, int64_t n_oct) {
     using S = DirectShape<TIn, E, L_>;
     constexpr int C = S::C, R = S::R, L = S::L, D = kDirectStages, EPC = S::EPC, CH = S::CH;
@@ -296,6 +343,7 @@ __global__ void __launch_bounds__(kDirectThreads)
     float* s_b1 = reinterpret_cast<float*>(lists + kDirectWarps);  // phase-1 key offsets, padded lane layout
     float* s_b2 = s_b1 + L * S::CS;                                // exact bias by expert
     uint64_t* bars = reinterpret_cast<uint64_t*>(s_b2 + E);
+    float* s_bmax = reinterpret_cast<float*>(bars + kDirectWarps * D);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -348,20 +396,26 @@ __global__ void __launch_bounds__(kDirectThreads)
             if (gw + d * nwarps < n_oct) issue(gw + d * nwarps, d);
     }
 
-    // Bias tables and the candidate band.  Every warp reads the whole bias
-    // (L2-resident) to find max |b|; warp w writes the entries e with
-    // (e / 32) % kDirectWarps == w.
+    // Bias tables and the candidate band: the block's threads share the
+    // entries (E / 128 each) and the per-warp maxima of |b| meet in shared
+    // memory.
     float bmax = 0.0f;
-    for (int e = lane; e < E; e += 32) {
-        const float b = BIAS ? bias_as_used(__ldg(a.bias + e), a.bias_bf16) : 0.0f;
-        bmax = fmaxf(bmax, fabsf(b));
-        if ((e / 32) % kDirectWarps == warp) {
+#pragma unroll
+    for (int e0 = 0; e0 < E; e0 += kDirectThreads) {
+        const int e = e0 + (int)threadIdx.x;
+        if (e < E) {
+            const float b = BIAS ? bias_as_used(__ldg(a.bias + e), a.bias_bf16) : 0.0f;
+            bmax = fmaxf(bmax, fabsf(b));
             s_b2[e] = b;
             s_b1[(e / C) * S::CS + e % C] = (MODE == kKeyApprox) ? 0.5f + b : b;
         }
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFullMask, bmax, o));
+    if (lane == 0) s_bmax[warp] = bmax;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kDirectWarps; ++w) bmax = fmaxf(bmax, s_bmax[w]);
     float band = 0.0f;
     if constexpr (MODE != kKeyRaw) {
         // eps = key error (tanh bound or pair/single difference) + 4 ulp of
@@ -369,7 +423,6 @@ __global__ void __launch_bounds__(kDirectThreads)
         const float round = (bmax + 2.0f) * (1.0f / 2097152.0f);
         band = (MODE == kKeyApprox) ? 2.0f * (0.5f * kTanhApproxErr + round) : 2.0f * (kPairKeyErr + round);
     }
-    __syncthreads();
 
     const int K = a.K;
     const float* b1 = s_b1 + sl * S::CS;
@@ -528,18 +581,26 @@ __global__ void __launch_bounds__(kDirectThreads)
                 const float* k8 = key + 8 * u;
                 bm[u] = fmax3(fmax3(k8[0], k8[1], k8[2]), fmax3(k8[3], k8[4], k8[5]), fmaxf(k8[6], k8[7]));
             }
-            // Each lane contributes its four largest block maxima (the 16 of
-            // the row are distinct experts, so their k-th largest is still a
-            // lower bound): two sorted halves, then the top four of the two.
-            float b4[4] = {bm[0], bm[1], bm[2], bm[3]};
-            if constexpr (S::NB > 4) {
-                float h[4] = {bm[4], bm[5], bm[6], bm[7]};
-                sort_desc(b4);
-                sort_desc(h);
+            if constexpr (L == 8 && S::NB == 4) {
+                // Eight lanes: each contributes its two largest block maxima
+                // (16 distinct experts per row, so their k-th largest is a
+                // lower bound).
+                const float ah = fmaxf(bm[0], bm[1]), al = fminf(bm[0], bm[1]);
+                const float ch = fmaxf(bm[2], bm[3]), cl = fminf(bm[2], bm[3]);
+                tau = row_kth2<L>(fmaxf(ah, ch), fmax3(fminf(ah, ch), al, cl), K, rowmax);
+            } else {
+                // Each lane contributes its four largest block maxima: two
+                // sorted halves, then the top four of the two.
+                float b4[4] = {bm[0], bm[1], bm[2], bm[3]};
+                if constexpr (S::NB > 4) {
+                    float h[4] = {bm[4], bm[5], bm[6], bm[7]};
+                    sort_desc(b4);
+                    sort_desc(h);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) b4[i] = fmaxf(b4[i], h[3 - i]);
+                    for (int i = 0; i < 4; ++i) b4[i] = fmaxf(b4[i], h[3 - i]);
+                }
+                tau = row_kth<4, L>(b4, K, rowmax);
             }
-            tau = row_kth<4, L>(b4, K, rowmax);
         }
         const float lo = tau - band;
 
@@ -591,58 +652,95 @@ __global__ void __launch_bounds__(kDirectThreads)
         }
         const int nf = (valid && !slow) ? n : 0;
         const int nmax = __reduce_max_sync(kFullMask, nf);
-        const int jmax = (nmax + 3) & ~3;
         __syncwarp();
         constexpr int TPL = kDirectCap / L;  // list entries per lane
         uint32_t kt[TPL];
         float pt[TPL];
         int it[TPL];
+        int rk[TPL];  // rank of the entry among the row's candidates
 #pragma unroll
         for (int u = 0; u < TPL; ++u) {
-            const int t = sl + u * L;
             kt[u] = 0u;
             pt[u] = 0.0f;
             it[u] = 0;
-            if (u * L < nmax) {  // warp-uniform bound
-                if (t < nf) {
-                    const int e = lst.id[rr][t];
-                    float kx, px;
-                    exact_key<SCORE, BIAS, MODE>(logit_at(e / C, e % C), BIAS ? s_b2[e] : 0.0f, kx, px);
-                    kt[u] = order_u32(kx);
-                    pt[u] = px;
-                    it[u] = e;
-                }
-                if (t < jmax) lst.key[rr][t] = kt[u];  // 0 pads the list to jmax
-            }
+            rk[u] = kDirectCap;
         }
-        __syncwarp();
-
+        // exact key of list entry t = sl + u * L (0 beyond the row's list)
+        auto entry_key = [&](int u) {
+            const int t = sl + u * L;
+            if (t < nf) {
+                const int e = lst.id[rr][t];
+                float kx, px;
+                exact_key<SCORE, BIAS, MODE>(logit_at(e / C, e % C), BIAS ? s_b2[e] : 0.0f, kx, px);
+                kt[u] = order_u32(kx);
+                pt[u] = px;
+                it[u] = e;
+            }
+        };
         // ---- rank by counting: slot of candidate t = #candidates above it ---
         // set.gt gives -1 per key above; three-input adds sum them.  The
         // winners (rank < K) go to the row's slot table.
+        auto count_above = [](const uint4& k4, uint32_t k0, int c) {
+            uint32_t s0, s1, s2, s3;
+            asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s0) : "r"(k4.x), "r"(k0));
+            asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s1) : "r"(k4.y), "r"(k0));
+            asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s2) : "r"(k4.z), "r"(k0));
+            asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s3) : "r"(k4.w), "r"(k0));
+            c = c - (int)s0 - (int)s1;
+            return c - (int)s2 - (int)s3;
+        };
         int rsum = 0;
+        if (L == 8 && nmax <= kDirectFastN) {
+            // Every row of the warp has at most 16 candidates (nearly all
+            // octets): the list is padded to 16 with zero keys, each lane
+            // keys 16 / L entries, then reads the 16 keys once and ranks its
+            // entries against them.
+            constexpr int FS = kDirectFastN / L;
 #pragma unroll
-        for (int u = 0; u < TPL; ++u) {
-            if (u * L < nmax) {  // warp-uniform bound
+            for (int u = 0; u < FS; ++u) {
+                entry_key(u);
+                lst.key[rr][sl + u * L] = kt[u];
+            }
+            __syncwarp();
+            uint4 k4[kDirectFastN / 4];
+#pragma unroll
+            for (int q = 0; q < kDirectFastN / 4; ++q) k4[q] = *reinterpret_cast<const uint4*>(&lst.key[rr][4 * q]);
+#pragma unroll
+            for (int u = 0; u < FS; ++u) {
                 const int t = sl + u * L;
                 const uint32_t k0 = t < nf ? kt[u] : 0xffffffffu;
                 int c = 0;
 #pragma unroll
-                for (int j4 = 0; j4 < kDirectCap; j4 += 4) {
-                    if (j4 < jmax) {
-                        const uint4 k4 = *reinterpret_cast<const uint4*>(&lst.key[rr][j4]);
-                        uint32_t s0, s1, s2, s3;
-                        asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s0) : "r"(k4.x), "r"(k0));
-                        asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s1) : "r"(k4.y), "r"(k0));
-                        asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s2) : "r"(k4.z), "r"(k0));
-                        asm("set.gt.u32.u32 %0, %1, %2;" : "=r"(s3) : "r"(k4.w), "r"(k0));
-                        c = c - (int)s0 - (int)s1;
-                        c = c - (int)s2 - (int)s3;
-                    }
-                }
+                for (int q = 0; q < kDirectFastN / 4; ++q) c = count_above(k4[q], k0, c);
                 if (t < nf) {
                     rsum += c;
-                    if (c < K) lst.out[rr][c] = make_float2(pt[u], __int_as_float(it[u]));
+                    rk[u] = c;
+                }
+            }
+        } else {
+            const int jmax = (nmax + 3) & ~3;
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) {
+                const int t = sl + u * L;
+                if (u * L < nmax) {  // warp-uniform bound
+                    entry_key(u);
+                    if (t < jmax) lst.key[rr][t] = kt[u];  // 0 pads the list to jmax
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) {
+                if (u * L < nmax) {  // warp-uniform bound
+                    const int t = sl + u * L;
+                    const uint32_t k0 = t < nf ? kt[u] : 0xffffffffu;
+                    int c = 0;
+#pragma unroll
+                    for (int j4 = 0; j4 < kDirectCap; j4 += 4)
+                        if (j4 < jmax) c = count_above(*reinterpret_cast<const uint4*>(&lst.key[rr][j4]), k0, c);
+                    if (t < nf) {
+                        rsum += c;
+                        rk[u] = c;
+                    }
                 }
             }
         }
@@ -653,7 +751,6 @@ __global__ void __launch_bounds__(kDirectThreads)
         // with a lower expert index counting as above.
         const bool ties = valid && !slow && rsum != n * (n - 1) / 2;
         if (__any_sync(kFullMask, ties)) {
-            __syncwarp();  // the first ranking's slot writes land before these
 #pragma unroll
             for (int u = 0; u < TPL; ++u) {
                 const int t = sl + u * L;
@@ -663,7 +760,7 @@ __global__ void __launch_bounds__(kDirectThreads)
                         const uint32_t kj = lst.key[rr][jj];
                         c += (kj > kt[u]) || (kj == kt[u] && lst.id[rr][jj] < it[u]);
                     }
-                    if (ties && t < nf && c < K) lst.out[rr][c] = make_float2(pt[u], __int_as_float(it[u]));
+                    if (ties && t < nf) rk[u] = c;
                 }
             }
         }
@@ -732,10 +829,15 @@ __global__ void __launch_bounds__(kDirectThreads)
                     }
                 }
             }
+            __syncwarp();
         }
-        __syncwarp();
 
-        // ---- weights: gather, renormalise, scale, store ----------------------
+        // ---- weights: renormalise, scale, store ------------------------------
+        // Each lane holds its list entries and their ranks: the entries ranked
+        // below k are the row's winners, stored at their rank.  Their sum runs
+        // over the lane's entries in list order, then across the row's lanes,
+        // so a row's weights depend on that row alone.  Rows routed by the
+        // whole warp take their winners from the slot table instead.
         float denom_all = 1.0f;
         if constexpr (SCORE == kSoftmax) {
             if (!a.renorm) {
@@ -747,37 +849,58 @@ __global__ void __launch_bounds__(kDirectThreads)
                 denom_all = s;
             }
         }
-        constexpr int SPL = (8 + L - 1) / L;  // output slots per lane
-        float wv[SPL];
-        int iv[SPL];
-        float wsum = 0.0f;
+        auto weight_of = [&](float p) { return (SCORE == kSoftmax) ? softmax_num(p, rowmax, a.softcap) : p; };
+        auto scale_of = [&](float wsum) {
 #pragma unroll
-        for (int v = 0; v < SPL; ++v) {
-            const int js = sl + v * L;
-            wv[v] = 0.0f;
-            iv[v] = 0;
-            if (js < K) {
-                const float2 o = lst.out[rr][js];
-                const float w = (SCORE == kSoftmax) ? softmax_num(o.x, rowmax, a.softcap) : o.x;
-                wv[v] = w;
-                iv[v] = __float_as_int(o.y);
-                wsum += w;
+            for (int o = 1; o < L; o <<= 1) wsum += __shfl_xor_sync(kFullMask, wsum, o);
+            if (a.renorm) return __fdividef(a.rsf, wsum);
+            return (SCORE == kSoftmax) ? __fdividef(a.rsf, denom_all) : a.rsf;
+        };
+        {
+            float wr[TPL];
+            float wsum = 0.0f;
+#pragma unroll
+            for (int u = 0; u < TPL; ++u) {
+                wr[u] = rk[u] < K ? weight_of(pt[u]) : 0.0f;
+                wsum += wr[u];
+            }
+            const float scale = scale_of(wsum);
+            if (valid && !slow) {
+#pragma unroll
+                for (int u = 0; u < TPL; ++u) {
+                    if (rk[u] < K) {
+                        a.weights[row * K + rk[u]] = wr[u] * scale;
+                        a.ids[row * K + rk[u]] = it[u];
+                    }
+                }
             }
         }
-#pragma unroll
-        for (int o = 1; o < L; o <<= 1) wsum += __shfl_xor_sync(kFullMask, wsum, o);
-        float scale;
-        if (a.renorm)
-            scale = __fdividef(a.rsf, wsum);
-        else
-            scale = (SCORE == kSoftmax) ? __fdividef(a.rsf, denom_all) : a.rsf;
-        if (valid) {
+        if (slow_rows) {
+            constexpr int SPL = (8 + L - 1) / L;  // output slots per lane
+            float wv[SPL];
+            int iv[SPL];
+            float wsum = 0.0f;
 #pragma unroll
             for (int v = 0; v < SPL; ++v) {
                 const int js = sl + v * L;
-                if (js < K) {
-                    a.weights[row * K + js] = wv[v] * scale;
-                    a.ids[row * K + js] = iv[v];
+                wv[v] = 0.0f;
+                iv[v] = 0;
+                if (slow && js < K) {
+                    const float2 o = lst.out[rr][js];
+                    wv[v] = weight_of(o.x);
+                    iv[v] = __float_as_int(o.y);
+                    wsum += wv[v];
+                }
+            }
+            const float scale = scale_of(wsum);
+            if (valid && slow) {
+#pragma unroll
+                for (int v = 0; v < SPL; ++v) {
+                    const int js = sl + v * L;
+                    if (js < K) {
+                        a.weights[row * K + js] = wv[v] * scale;
+                        a.ids[row * K + js] = iv[v];
+                    }
                 }
             }
         }
