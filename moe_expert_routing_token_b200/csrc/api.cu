@@ -370,11 +370,16 @@ int try_direct_e(const RouteArgs& a, cudaStream_t st) {
     return try_direct_el<TIn, E, 8, SCORE, BIAS>(a, st);
 }
 
+// Above this many rows the two-phase streaming kernel, whose ring keeps every
+// SM busy for the whole call, issues fewer instructions per row and wins.
+// Measured on B200 (bf16 E = 256, k = 8): 33.9 against 36.9 us at M = 131072
+// and 58.8 against 69.2 at 262144 (sigmoid with bias); grouped (G = 8,
+// TG = 4) 40.0 against 50.3 and 70.2 against 96.8.
+constexpr int64_t kDirectMaxRows = 65536;
+
 template <typename TIn, int SCORE, bool BIAS>
 int try_direct(const RouteArgs& a, cudaStream_t st) {
-    if (a.K > 8 || !aligned(a.logits, 16)) return -1;
-    // TMA box coordinates are 32-bit: (M * 8) rows of 128 bytes at most
-    if (a.M > (int64_t(1) << 28)) return -1;
+    if (a.K > 8 || !aligned(a.logits, 16) || a.M > kDirectMaxRows) return -1;
     // E = 160 (rows staged by per-row copies) measured slower than the
     // two-phase streaming kernel at every size it would serve (fp32, k = 6,
     // G = 8: 15.8 against 9.7 us at M = 16384), so it is left to that kernel.

@@ -241,36 +241,6 @@ __device__ __forceinline__ float row_kth(const float (&in)[P], int K, float& vma
     return kth_of_sorted8(a, K);
 }
 
-// As row_kth for eight lanes holding two values each, t0 >= t1: the xor-1
-// exchange makes sorted 4-lists ([t0, t1, p1, p0] is bitonic), the xor-2
-// exchange sorted 8-lists, and the xor-4 exchange the top 8 of the 16 (the
-// elementwise maximum against the reversed partner, a bitonic sequence that
-// is sorted only when K < 8 needs it).
-template <int L>
-__device__ __forceinline__ float row_kth2(float t0, float t1, int K, float& vmax) {
-    static_assert(L == 8, "two values per lane on eight lanes");
-    float a[8];
-    {
-        float x[4] = {t0, t1, __shfl_xor_sync(kFullMask, t1, 1), __shfl_xor_sync(kFullMask, t0, 1)};
-        bitonic_clean_desc(x);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            a[i] = x[i];
-            a[7 - i] = __shfl_xor_sync(kFullMask, x[i], 2);
-        }
-        bitonic_clean_desc(a);
-        float b[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = __shfl_xor_sync(kFullMask, a[i], 4);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], b[7 - i]);
-    }
-    vmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-    if (K == 8) return fminf(fminf(fminf(a[0], a[1]), fminf(a[2], a[3])), fminf(fminf(a[4], a[5]), fminf(a[6], a[7])));
-    bitonic_clean_desc(a);
-    return kth_of_sorted8(a, K);
-}
-
 // Unpack one 16-byte chunk into fp32 values.
 template <typename TIn>
 __device__ __forceinline__ void unpack_chunk(const uint4& v, float* x);
@@ -657,13 +627,11 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
         uint32_t kt[TPL];
         float pt[TPL];
         int it[TPL];
-        int rk[TPL];  // rank of the entry among the row's candidates
 #pragma unroll
         for (int u = 0; u < TPL; ++u) {
             kt[u] = 0u;
             pt[u] = 0.0f;
             it[u] = 0;
-            rk[u] = kDirectCap;
         }
         // exact key of list entry t = sl + u * L (0 beyond the row's list)
         auto entry_key = [&](int u) {
@@ -714,7 +682,7 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
                 for (int q = 0; q < kDirectFastN / 4; ++q) c = count_above(k4[q], k0, c);
                 if (t < nf) {
                     rsum += c;
-                    rk[u] = c;
+                    if (c < K) lst.out[rr][c] = make_float2(pt[u], __int_as_float(it[u]));
                 }
             }
         } else {
@@ -739,7 +707,7 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
                         if (j4 < jmax) c = count_above(*reinterpret_cast<const uint4*>(&lst.key[rr][j4]), k0, c);
                     if (t < nf) {
                         rsum += c;
-                        rk[u] = c;
+                        if (c < K) lst.out[rr][c] = make_float2(pt[u], __int_as_float(it[u]));
                     }
                 }
             }
@@ -751,6 +719,7 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
         // with a lower expert index counting as above.
         const bool ties = valid && !slow && rsum != n * (n - 1) / 2;
         if (__any_sync(kFullMask, ties)) {
+            __syncwarp();  // the first ranking's slot writes land before these
 #pragma unroll
             for (int u = 0; u < TPL; ++u) {
                 const int t = sl + u * L;
@@ -760,7 +729,7 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
                         const uint32_t kj = lst.key[rr][jj];
                         c += (kj > kt[u]) || (kj == kt[u] && lst.id[rr][jj] < it[u]);
                     }
-                    if (ties && t < nf) rk[u] = c;
+                    if (ties && t < nf && c < K) lst.out[rr][c] = make_float2(pt[u], __int_as_float(it[u]));
                 }
             }
         }
@@ -829,15 +798,12 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
                     }
                 }
             }
-            __syncwarp();
         }
+        __syncwarp();
 
-        // ---- weights: renormalise, scale, store ------------------------------
-        // Each lane holds its list entries and their ranks: the entries ranked
-        // below k are the row's winners, stored at their rank.  Their sum runs
-        // over the lane's entries in list order, then across the row's lanes,
-        // so a row's weights depend on that row alone.  Rows routed by the
-        // whole warp take their winners from the slot table instead.
+        // ---- weights: gather from the slot table, renormalise, scale, store --
+        // Lane sl takes output slot sl (and sl + L, ...): the sum runs over the
+        // slots in a fixed order, so a row's weights depend on that row alone.
         float denom_all = 1.0f;
         if constexpr (SCORE == kSoftmax) {
             if (!a.renorm) {
@@ -857,25 +823,6 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
             return (SCORE == kSoftmax) ? __fdividef(a.rsf, denom_all) : a.rsf;
         };
         {
-            float wr[TPL];
-            float wsum = 0.0f;
-#pragma unroll
-            for (int u = 0; u < TPL; ++u) {
-                wr[u] = rk[u] < K ? weight_of(pt[u]) : 0.0f;
-                wsum += wr[u];
-            }
-            const float scale = scale_of(wsum);
-            if (valid && !slow) {
-#pragma unroll
-                for (int u = 0; u < TPL; ++u) {
-                    if (rk[u] < K) {
-                        a.weights[row * K + rk[u]] = wr[u] * scale;
-                        a.ids[row * K + rk[u]] = it[u];
-                    }
-                }
-            }
-        }
-        if (slow_rows) {
             constexpr int SPL = (8 + L - 1) / L;  // output slots per lane
             float wv[SPL];
             int iv[SPL];
@@ -885,7 +832,7 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
                 const int js = sl + v * L;
                 wv[v] = 0.0f;
                 iv[v] = 0;
-                if (slow && js < K) {
+                if (js < K) {
                     const float2 o = lst.out[rr][js];
                     wv[v] = weight_of(o.x);
                     iv[v] = __float_as_int(o.y);
@@ -893,7 +840,7 @@ __global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCO
                 }
             }
             const float scale = scale_of(wsum);
-            if (valid && slow) {
+            if (valid) {
 #pragma unroll
                 for (int v = 0; v < SPL; ++v) {
                     const int js = sl + v * L;

@@ -450,10 +450,11 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                     const float* k8 = key + 8 * (u % (C / 8));
                     q[u] = fmax3(fmax3(k8[0], k8[1], k8[2]), fmax3(k8[3], k8[4], k8[5]), fmaxf(k8[6], k8[7]));
                 }
-                float top[8];
-                segment_top8_of4<L>(q, top);
-                m1 = top[0];  // row max (all lanes)
-                tau = kth_of_sorted8(top, K);
+                // the lane's two largest quarter maxima: the K-th largest of
+                // the row's 16 is still a lower bound (distinct experts)
+                const float ah = fmaxf(q[0], q[1]), al = fminf(q[0], q[1]);
+                const float ch = fmaxf(q[2], q[3]), cl = fminf(q[2], q[3]);
+                tau = row_kth2<L>(fmaxf(ah, ch), fmax3(fminf(ah, ch), al, cl), K, m1);  // m1: row max
             } else {
                 top2_of(key, m1, m2);
             }
