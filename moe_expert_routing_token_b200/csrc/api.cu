@@ -294,11 +294,14 @@ int launch_direct(const RouteArgs& a, cudaStream_t st) {
 }
 
 // Batches up to this size route one row per warp (route_warp_kernel): the
-// shortest chain per row.  Measured on B200 (bf16 E = 256, k = 8, sigmoid
-// with bias): 2.1 us at M = 64 and 4.7 us at M = 4096 (direct kernel: 4.3
-// and 5.8 us); from M = 8192 the direct kernel's fewer instructions per row
-// win (5.9 against 8.2 us).
+// shortest chain per row.  Where the direct kernel takes the shape (E = 256,
+// k <= 8, every group kept or 8 groups) it takes over above 3072 rows:
+// measured on B200 (bf16 E = 256, k = 8, sigmoid with bias), the warp-per-row
+// kernel takes 2.1 / 2.5 / 3.1 us at M = 256 / 1024 / 2048 against 2.8 / 3.4
+// / 3.5 for the direct kernel, and 4.7 against 4.4 us at M = 4096 (grouped,
+// G = 8: 5.3 against 4.8).
 constexpr int64_t kWarpRowMaxRows = 4096;
+constexpr int64_t kWarpRowMaxRowsBeforeDirect = 3072;
 
 template <typename TIn, int E, int SCORE, bool BIAS, bool GROUPED>
 int launch_warp_rows(const RouteArgs& a, cudaStream_t st) {
@@ -337,7 +340,9 @@ int try_warp_rows_e(const RouteArgs& a, cudaStream_t st) {
 
 template <typename TIn, int SCORE, bool BIAS>
 int try_warp_rows(const RouteArgs& a, cudaStream_t st) {
-    if (a.M > kWarpRowMaxRows || 32 % a.G != 0) return -1;
+    // the shapes try_direct takes (below its row limit)
+    const bool direct_shape = a.E == 256 && a.K <= 8 && (a.TG == a.G || a.G == 8) && aligned(a.logits, 16);
+    if (a.M > (direct_shape ? kWarpRowMaxRowsBeforeDirect : kWarpRowMaxRows) || 32 % a.G != 0) return -1;
     if (a.E == 256) return try_warp_rows_e<TIn, 256, SCORE, BIAS>(a, st);
     if (a.E == 160) return try_warp_rows_e<TIn, 160, SCORE, BIAS>(a, st);
     return -1;

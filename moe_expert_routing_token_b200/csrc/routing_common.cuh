@@ -280,35 +280,33 @@ __device__ __forceinline__ float kth_of_sorted8(const float (&top)[8], int K) {
     return t;
 }
 
-// The K-th largest (1 <= K <= 8) and the largest of the 16 values held two
-// per lane, t0 >= t1, by the eight lanes of a row: the xor-1
-// exchange makes sorted 4-lists ([t0, t1, p1, p0] is bitonic), the xor-2
-// exchange sorted 8-lists, and the xor-4 exchange the top 8 of the 16 (the
-// elementwise maximum against the reversed partner, a bitonic sequence that
-// is sorted only when K < 8 needs it).
+// As segment_top8, each lane contributing four values (any order): sort
+// them, merge with the xor-1 partner into a sorted 8, then keep the top 8
+// over the xor-2 and xor-4 partners.
 template <int L>
-__device__ __forceinline__ float row_kth2(float t0, float t1, int K, float& vmax) {
-    static_assert(L == 8, "two values per lane on eight lanes");
+__device__ __forceinline__ void segment_top8_of4(const float (&q)[4], float (&out)[8]) {
+    static_assert(L == 8, "eight lanes per segment");
     float a[8];
-    {
-        float x[4] = {t0, t1, __shfl_xor_sync(kFullMask, t1, 1), __shfl_xor_sync(kFullMask, t0, 1)};
-        bitonic_clean_desc(x);
+    a[0] = q[0]; a[1] = q[1]; a[2] = q[2]; a[3] = q[3];
+    cx_desc(a[0], a[1]);
+    cx_desc(a[2], a[3]);
+    cx_desc(a[0], a[2]);
+    cx_desc(a[1], a[3]);
+    cx_desc(a[1], a[2]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            a[i] = x[i];
-            a[7 - i] = __shfl_xor_sync(kFullMask, x[i], 2);
-        }
-        bitonic_clean_desc(a);
+    for (int i = 0; i < 4; ++i) a[7 - i] = __shfl_xor_sync(kFullMask, a[i], 1);
+    bitonic_clean_desc(a);
+#pragma unroll
+    for (int o = 2; o < L; o <<= 1) {
         float b[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = __shfl_xor_sync(kFullMask, a[i], 4);
+        for (int i = 0; i < 8; ++i) b[i] = __shfl_xor_sync(kFullMask, a[i], o);
 #pragma unroll
         for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], b[7 - i]);
+        bitonic_clean_desc(a);
     }
-    vmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-    if (K == 8) return fminf(fminf(fminf(a[0], a[1]), fminf(a[2], a[3])), fminf(fminf(a[4], a[5]), fminf(a[6], a[7])));
-    bitonic_clean_desc(a);
-    return kth_of_sorted8(a, K);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = a[i];
 }
 
 template <typename T>

@@ -56,6 +56,7 @@
 #pragma once
 
 #include "routing_common.cuh"
+#include "routing_threshold.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {

@@ -9,7 +9,8 @@
 //  * Phase 1 (a team of 8 warps, 8 lanes per row, C experts per lane): the
 //    lane scores its C experts, takes its top-2, the row's kept groups and a
 //    threshold tau that the k-th best admissible key is known to reach (the
-//    k-th largest of the kept lanes' top-2 values), and writes one bitmask
+//    k-th largest of the kept lanes' top-2 values, or with every group kept
+//    of each lane's two largest 8-expert quarter maxima), and writes one bitmask
 //    word per lane - its experts with key >= tau - band - to a per-block
 //    table.  No compaction and no ranking here.  Two teams take alternate
 //    blocks.
@@ -38,6 +39,7 @@
 #pragma once
 
 #include "routing_staged.cuh"
+#include "routing_threshold.cuh"
 
 namespace moe {
 
@@ -443,7 +445,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
             const bool quarters = (C == 32) && all_groups;
             if (quarters) {
                 // every group kept: the threshold comes from the maxima of the
-                // lane's four 8-expert quarters (32 distinct experts per row)
+                // lane's four 8-expert quarters (distinct experts)
                 float q[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {

@@ -1,7 +1,7 @@
-"""Parity of the direct routing kernel (E = 256, k <= 8, batches above 4096
+"""Parity of the direct routing kernel (E = 256, k <= 8, batches above 3072
 rows) against the oracle, element by element (GPU only).
 
-Batches of more than 4096 rows with E = 256 and every group kept, or eight
+Batches of more than 3072 rows with E = 256 and every group kept, or eight
 groups, take the direct kernel: eight lanes per row, a threshold from block
 maxima, candidates ranked by counting.  The cases cover its key modes
 (approximate sigmoid keys, exact grouped keys, raw logits), k = 8 and the
@@ -36,7 +36,7 @@ SHAPES = [
 
 @pytest.mark.parametrize("op,G,TG,k,renorm,rsf,use_bias", SHAPES)
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("M", [4099, 9001])
+@pytest.mark.parametrize("M", [3073, 4099, 9001])
 def test_direct_shapes(op, G, TG, k, renorm, rsf, use_bias, dtype, M):
     x = inputs.random_logits(M, 256, 2.0, dtype, seed=M + 13 * G + k)
     bias = inputs.random_bias(256, 0.05, seed=G + k) if use_bias else None
