@@ -81,3 +81,20 @@ def test_equal_rows_pick_lowest_indices(op, G, TG, k):
     orc = run_oracle(op, x, None, k, True, G, TG, 1.0)
     assert np.array_equal(ids[::9], orc.ids[::9])
     check(op, x, None, k, True, G, TG, 1.0)
+
+
+# fp32 E = 160, eight groups of 20 (one lane each when grouped)
+SHAPES_160 = [
+    ("softmax", 8, 3, 6, False, 1.0, False),  # grouped softmax, the full denominator (DeepSeek-V2)
+    ("softmax", 1, 1, 6, True, 1.0, False),   # raw logits
+    ("sigmoid", 8, 4, 8, True, 2.5, True),    # grouped, exact keys
+    ("sigmoid", 1, 1, 4, True, 1.0, True),    # approximate keys, k = 4
+]
+
+
+@pytest.mark.parametrize("op,G,TG,k,renorm,rsf,use_bias", SHAPES_160)
+@pytest.mark.parametrize("M", [5003, 9001])
+def test_e160_fp32_shapes(op, G, TG, k, renorm, rsf, use_bias, M):
+    x = inputs.random_logits(M, 160, 1.5, torch.float32, seed=M + 7 * G + k)
+    bias = inputs.random_bias(160, 0.05, seed=G + k + 1) if use_bias else None
+    check(op, x, bias, k, renorm, G, TG, rsf)
