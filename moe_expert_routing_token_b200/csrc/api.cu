@@ -381,14 +381,18 @@ int try_direct_e(const RouteArgs& a, cudaStream_t st) {
 // and 58.8 against 69.2 at 262144 (sigmoid with bias); grouped (G = 8,
 // TG = 4) 40.0 against 50.3 and 70.2 against 96.8.
 constexpr int64_t kDirectMaxRows = 65536;
+constexpr int64_t kDirectMaxRows160 = 16384;
 
 template <typename TIn, int SCORE, bool BIAS>
 int try_direct(const RouteArgs& a, cudaStream_t st) {
     if (a.K > 8 || !aligned(a.logits, 16) || a.M > kDirectMaxRows) return -1;
-    // E = 160 (rows staged by per-row copies) measured slower than the
-    // two-phase streaming kernel at every size it would serve (fp32, k = 6,
-    // G = 8: 15.8 against 9.7 us at M = 16384), so it is left to that kernel.
     if (a.E == 256) return try_direct_e<TIn, 256, SCORE, BIAS>(a, st);
+    // fp32 E = 160 (rows staged by per-row copies, 20 experts per lane) up to
+    // 16384 rows; above, the two-phase streaming kernel.  Measured on B200
+    // (softmax, G = 8, TG = 3, k = 6): 5.7 / 9.3 / 15.0 us at M = 8192 /
+    // 16384 / 32768 against 7.7 / 9.6 / 13.8 for the streaming kernel.
+    if constexpr (sizeof(TIn) == 4)
+        if (a.E == 160 && a.M <= kDirectMaxRows160) return try_direct_e<TIn, 160, SCORE, BIAS>(a, st);
     return -1;
 }
 

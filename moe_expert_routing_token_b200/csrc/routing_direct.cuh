@@ -17,17 +17,17 @@
 //    those rows, and the swizzle spreads the lanes of a row (and the rows
 //    of a quarter-warp) over distinct bank groups.  For E = 160 each
 //    row is copied to a padded shared-memory row (or the octet in one copy
-//    when no padding is needed), which spreads the banks the same way (that
-//    shape is built and correct, but the library dispatches E = 160 to the
-//    two-phase streaming kernel, which measured faster).  The register order
-//    of every lane's experts is its segment order.
+//    when no padding is needed), which spreads the banks the same way (the
+//    library takes that shape for fp32 rows, 20 experts per lane).  The
+//    register order of every lane's experts is its segment order.
 //  * Threshold.  Each lane scores its C experts (selection keys), takes the
-//    maxima of blocks of 8 experts, and the row's L lanes find tau, the
-//    k-th largest of each lane's two (L = 8) or four (L = 4) largest block
-//    maxima, with a merge network over xor-shuffles: tau is a lower bound
-//    for the k-th best key, since the maxima belong to distinct experts.
-//    With group selection the kept groups are ranked first and tau is the
-//    k-th largest of their block maxima.
+//    maxima of blocks of 8 experts (the first 16 of 20 with E = 160; blocks
+//    of a quarter of a group when groups are selected), and the row's L
+//    lanes find tau, the k-th largest of each lane's two (L = 8) or four
+//    (L = 4) largest block maxima, with a merge network over xor-shuffles:
+//    tau is a lower bound for the k-th best key, since the maxima belong to
+//    distinct experts.  With group selection the kept groups are ranked
+//    first and tau is the k-th largest of their block maxima.
 //  * Candidates.  Experts with key >= tau - band (about 10 per row on the
 //    benchmark workloads) are appended to a per-row list; the row's L
 //    lanes then share the list evenly, compute the exact keys of their
@@ -128,7 +128,7 @@ struct DirectShape {
     static constexpr int STAGE = R * RS;             // bytes per staged octet (a multiple of 1024 for TMA)
     static constexpr int NB = C / 8;                 // blocks of 8 experts per lane
     static constexpr int MW = (C + 31) / 32;         // candidate mask words per lane
-    static_assert((L == 4 || L == 8) && E % L == 0 && SEG % 16 == 0 && C % 8 == 0 && 8 % EPC == 0,
+    static_assert((L == 4 || L == 8) && E % L == 0 && SEG % 16 == 0 && C % 4 == 0 && 8 % EPC == 0,
                   "unsupported direct shape");
     static_assert(RS > 0 && RS % 16 == 0, "no conflict-free staging layout");
     static_assert(!TMA || STAGE % 1024 == 0, "swizzled stages start on 1024-byte boundaries");
@@ -289,16 +289,17 @@ __device__ __forceinline__ void exact_key(float x, float b, float& key, float& p
 // Resident blocks per SM the compiler is asked to fit, the most that compile
 // without spills.  Eight lanes per bf16 row: 8 (64 registers) for
 // approximate keys, 7 (72) for the other sigmoid keys, 5 (96) for softmax;
-// at 16384 rows that puts (nearly) one octet per warp in flight.  Other
-// shapes: 4 (128 registers).
-template <typename TIn, int L, int SCORE, int MODE>
+// at 16384 rows that puts (nearly) one octet per warp in flight.  fp32
+// E = 160: 5 (96).  Other shapes: 4 (128 registers).
+template <typename TIn, int E, int L, int SCORE, int MODE>
 constexpr int direct_min_blocks() {
-    if (sizeof(TIn) != 2 || L != 8) return 4;
+    if (L != 8) return 4;
+    if (sizeof(TIn) != 2) return E == 160 ? 5 : 4;
     return SCORE == kSoftmax ? 5 : (MODE == kKeyApprox ? 8 : 7);
 }
 
 template <typename TIn, int E, int L_, int SCORE, bool BIAS, int MODE, int GS>
-__global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, L_, SCORE, MODE>())
+__global__ void __launch_bounds__(kDirectThreads, direct_min_blocks<TIn, E, L_, SCORE, MODE>())
     route_direct_kernel(const __grid_constant__ CUtensorMap tmap, RouteArgs a, int64_t n_oct) {
     using S = DirectShape<TIn, E, L_>;
     constexpr int C = S::C, R = S::R, L = S::L, D = kDirectStages, EPC = S::EPC, CH = S::CH;

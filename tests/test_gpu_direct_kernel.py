@@ -1,5 +1,6 @@
 """Parity of the direct routing kernel (E = 256, k <= 8, batches above 3072
-rows) against the oracle, element by element (GPU only).
+rows; fp32 E = 160 above 4096 rows) against the oracle, element by element
+(GPU only).
 
 Batches of more than 3072 rows with E = 256 and every group kept, or eight
 groups, take the direct kernel: eight lanes per row, a threshold from block
