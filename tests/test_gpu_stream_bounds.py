@@ -112,7 +112,7 @@ def _close_key_rows(M, E, n_close, dtype, seed):
 @pytest.mark.parametrize("G,TG", [(1, 1), (8, 4), (8, 8)])
 @pytest.mark.parametrize("bias_std", [0.0, 2e-5])
 def test_close_keys_beyond_the_approximation(dtype, G, TG, bias_std):
-    M, E, k = 2048, 256, 8   # large enough for the streaming kernel
+    M, E, k = 2048, 256, 8   # the warp-per-row kernel (larger batches below)
     x = _close_key_rows(M, E, 24, dtype, seed=G * 10 + TG)
     bias = inputs.random_bias(E, bias_std, seed=5) if bias_std else torch.zeros(E)
     check("sigmoid", x, bias, k, True, G, TG, 2.5)
@@ -149,3 +149,32 @@ def test_inputs_written_by_the_previous_kernel():
         w_ref, ids_ref = moe.biased_grouped_topk(pool[i].clone(), bias, k, True, 1, 1, 1.0)
         torch.cuda.synchronize()
         assert torch.equal(ids, ids_ref) and torch.equal(w, w_ref)
+
+
+# The sizes and shapes that reach the two-phase streaming kernel: E = 256
+# above 65536 rows, fp32 E = 160 above 16384 rows, bf16 E = 160 and E = 256
+# with groups dropped out of 2 or 4 above 4096 rows.
+STREAM_CASES = [
+    ("sigmoid", 256, 1, 1, 8, True, 1.0, True, torch.bfloat16, 65603),
+    ("sigmoid", 256, 8, 4, 8, True, 2.5, True, torch.bfloat16, 65603),
+    ("softmax", 160, 8, 3, 6, False, 1.0, False, torch.float32, 16411),
+    ("softmax", 160, 8, 3, 6, False, 1.0, False, torch.bfloat16, 5003),
+    ("sigmoid", 256, 4, 2, 6, True, 1.0, True, torch.bfloat16, 5003),
+    ("sigmoid", 256, 2, 1, 7, True, 1.0, True, torch.float32, 5003),
+]
+
+
+@pytest.mark.parametrize("op,E,G,TG,k,renorm,rsf,use_bias,dtype,M", STREAM_CASES)
+def test_streaming_kernel_sizes(op, E, G, TG, k, renorm, rsf, use_bias, dtype, M):
+    x = inputs.random_logits(M, E, 2.0, dtype, seed=M + E + G)
+    bias = inputs.random_bias(E, 0.05, seed=E + G) if use_bias else None
+    check(op, x, bias, k, renorm, G, TG, rsf)
+
+
+@pytest.mark.parametrize("G,TG", [(1, 1), (8, 4)])
+def test_close_keys_streaming_sizes(G, TG):
+    """Rows of close keys (as above) in a batch the streaming kernel takes."""
+    M, E, k = 65603, 256, 8
+    x = _close_key_rows(M, E, 24, torch.bfloat16, seed=G * 10 + TG + 1)
+    bias = inputs.random_bias(E, 2e-5, seed=5)
+    check("sigmoid", x, bias, k, True, G, TG, 2.5)
