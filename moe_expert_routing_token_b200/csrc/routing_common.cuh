@@ -280,35 +280,6 @@ __device__ __forceinline__ float kth_of_sorted8(const float (&top)[8], int K) {
     return t;
 }
 
-// As segment_top8, each lane contributing four values (any order): sort
-// them, merge with the xor-1 partner into a sorted 8, then keep the top 8
-// over the xor-2 and xor-4 partners.
-template <int L>
-__device__ __forceinline__ void segment_top8_of4(const float (&q)[4], float (&out)[8]) {
-    static_assert(L == 8, "eight lanes per segment");
-    float a[8];
-    a[0] = q[0]; a[1] = q[1]; a[2] = q[2]; a[3] = q[3];
-    cx_desc(a[0], a[1]);
-    cx_desc(a[2], a[3]);
-    cx_desc(a[0], a[2]);
-    cx_desc(a[1], a[3]);
-    cx_desc(a[1], a[2]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[7 - i] = __shfl_xor_sync(kFullMask, a[i], 1);
-    bitonic_clean_desc(a);
-#pragma unroll
-    for (int o = 2; o < L; o <<= 1) {
-        float b[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = __shfl_xor_sync(kFullMask, a[i], o);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], b[7 - i]);
-        bitonic_clean_desc(a);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) out[i] = a[i];
-}
-
 template <typename T>
 __device__ __forceinline__ float load_scalar(const T* p);
 template <>

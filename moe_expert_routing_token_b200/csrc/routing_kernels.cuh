@@ -30,6 +30,7 @@
 #pragma once
 
 #include "routing_common.cuh"
+#include "routing_threshold.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
@@ -176,9 +177,14 @@ struct SegRouter {
         } else if (K <= 8) {
             // Tighter: the K-th largest of all kept lanes' top-2 values (those
             // are K distinct kept experts).
-            float top[8];
-            segment_top8<L>(gsel ? m1 : -INFINITY, gsel ? m2 : -INFINITY, top);
-            tau = kth_of_sorted8(top, K);
+            if constexpr (L == 8) {
+                float vmax;
+                tau = row_kth2<L>(gsel ? m1 : -INFINITY, gsel ? m2 : -INFINITY, K, vmax);
+            } else {
+                float top[8];
+                segment_top8<L>(gsel ? m1 : -INFINITY, gsel ? m2 : -INFINITY, top);
+                tau = kth_of_sorted8(top, K);
+            }
         } else {
             const float my = gsel ? m2 : -INFINITY;
             int r = 0;

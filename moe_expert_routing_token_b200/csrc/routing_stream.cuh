@@ -490,9 +490,14 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 for (int o = L / 2; o >= 1; o >>= 1) v = fminf(v, __shfl_xor_sync(kFullMask, v, o));
                 tau = v;
             } else {
-                float top[8];
-                segment_top8<L>(gsel ? m1 : -INFINITY, gsel ? m2 : -INFINITY, top);
-                tau = kth_of_sorted8(top, K);
+                if constexpr (L == 8) {
+                    float vmax;
+                    tau = row_kth2<L>(gsel ? m1 : -INFINITY, gsel ? m2 : -INFINITY, K, vmax);
+                } else {
+                    float top[8];
+                    segment_top8<L>(gsel ? m1 : -INFINITY, gsel ? m2 : -INFINITY, top);
+                    tau = kth_of_sorted8(top, K);
+                }
             }
             const float lo = tau - band;
 
