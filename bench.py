@@ -658,14 +658,16 @@ def run_ours(args):
 def e2e_measure(name, M, sp, d, dev, stream, world, args):
     """Host-resident inputs: per step H2D of the logits (or hidden states) from
     pinned memory (in row-chunks on parallel copy streams), the C-ABI call,
-    D2H of weights and ids into pinned memory."""
+    D2H of weights and ids into pinned memory.  Consecutive steps overlap as
+    a serving loop would: step i + 1's input crosses PCIe into the second of
+    two device buffers while step i is routed and its outputs are read back."""
     import torch
     import torch.distributed as dist
 
     from moe_expert_routing_token_b200 import routing
     steps = max(1, min(args.steps, 200))
     src = (d["hidden"] if name in ("fused", "top1") else d["logits"]).pin_memory()
-    x = torch.empty_like(src, device=dev)
+    xs = [torch.empty_like(src, device=dev) for _ in range(2)]
     wgt = d["weight"].to(dev) if name in ("fused", "top1") else None
     bias = d["bias"].to(dev) if d["bias"] is not None else None
     w = torch.empty(M, sp.topk, dtype=torch.float32, device=dev)
@@ -676,24 +678,29 @@ def e2e_measure(name, M, sp, d, dev, stream, world, args):
     wsp = torch.zeros(max(1, need), dtype=torch.uint8, device=dev)
 
     # The step's input crosses PCIe as n_chunks row-chunks on their own
-    # streams: one 8 MiB pinned copy moved 12 GB/s on the B200 boxes, four
+    # streams: one 8 MiB pinned copy moved 12 GB/s on some B200 boxes, four
     # concurrent ones 47 GB/s.
     n_chunks = 4
     rows = src.shape[0]
     bounds = [rows * c // n_chunks for c in range(n_chunks + 1)]
     copy_streams = [torch.cuda.Stream(device=dev) for _ in range(n_chunks)]
-    copied = [torch.cuda.Event() for _ in range(n_chunks)]
+    copied = [[torch.cuda.Event() for _ in range(n_chunks)] for _ in range(2)]
+    read = [torch.cuda.Event() for _ in range(2)]  # the last call that read buffer b is done
+    count = [0]
 
     def step():
+        b = count[0] % 2
+        count[0] += 1
+        x = xs[b]
         cur = torch.cuda.current_stream()
         for c in range(n_chunks):
             cs = copy_streams[c]
-            cs.wait_stream(cur)  # the previous step has finished reading x
+            cs.wait_event(read[b])  # the call two steps back has finished reading this buffer
             with torch.cuda.stream(cs):
                 x[bounds[c]:bounds[c + 1]].copy_(src[bounds[c]:bounds[c + 1]], non_blocking=True)
-                copied[c].record(cs)
+                copied[b][c].record(cs)
         for c in range(n_chunks):
-            cur.wait_event(copied[c])
+            cur.wait_event(copied[b][c])
         if name == "fused":
             routing.fused_router_topk(x, wgt, bias, sp.topk, sp.renormalize, sp.num_expert_group,
                                       sp.topk_group, sp.routed_scaling_factor, workspace=wsp,
@@ -706,6 +713,7 @@ def e2e_measure(name, M, sp, d, dev, stream, world, args):
         else:
             routing.biased_grouped_topk(x, bias, sp.topk, sp.renormalize, sp.num_expert_group,
                                         sp.topk_group, sp.routed_scaling_factor, out=(w, ids))
+        read[b].record(cur)
         hw.copy_(w, non_blocking=True)
         hi.copy_(ids, non_blocking=True)
 
