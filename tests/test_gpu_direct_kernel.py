@@ -99,3 +99,19 @@ def test_e160_fp32_shapes(op, G, TG, k, renorm, rsf, use_bias, M):
     x = inputs.random_logits(M, 160, 1.5, torch.float32, seed=M + 7 * G + k)
     bias = inputs.random_bias(160, 0.05, seed=G + k + 1) if use_bias else None
     check(op, x, bias, k, renorm, G, TG, rsf)
+
+
+@pytest.mark.parametrize("n_close,every", [(20, 1), (40, 3)])
+@pytest.mark.parametrize("op,G,TG,k", [("softmax", 8, 3, 6), ("sigmoid", 1, 1, 8)])
+def test_e160_crowded_rows(n_close, every, op, G, TG, k):
+    """fp32 E = 160 rows with 20 or 40 experts close together: the general
+    list path and the whole-warp path of the 20-experts-per-lane form."""
+    M, E = 6007, 160
+    gen = torch.Generator().manual_seed(n_close + every + G)
+    x = torch.randn(M, E, generator=gen) * 1.5
+    rows = torch.arange(0, M, every)
+    idx = torch.stack([torch.randperm(E, generator=gen)[:n_close] for _ in range(len(rows))])
+    vals = 6.5 + 2.0 * torch.rand(len(rows), n_close, generator=gen)
+    x[rows] = x[rows].scatter(1, idx, vals)
+    bias = inputs.random_bias(E, 2e-5, seed=4) if op == "sigmoid" else None
+    check(op, x, bias, k, True, G, TG, 1.0)
